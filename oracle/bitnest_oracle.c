@@ -1,0 +1,229 @@
+/*
+ * BitNest nested W4/W8 linear layer: plain CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header, table or constant with
+ * the CUDA library.
+ *
+ * Every routine is the plainest reading of the "BitNest-Llama-3-8B" model
+ * card (the only page that fixes the arithmetic):
+ *   - section "Files", planes.safetensors entry: the plane layout (uint8
+ *     [N, K/2], unsigned nibbles u = q + 8, byte j holds column 2j in its low
+ *     nibble and column 2j+1 in its high nibble), the fp16 group scales
+ *     [N, K/128] and the two dequantisation formulas
+ *         draft  W4 = (hi - 8) * scale
+ *         target W8 = (16 * (hi - 8) + (lo - 8)) * scale / 16 ;
+ *   - the model table, row "Activations": symmetric int8 per token, per
+ *     128-column group for o_proj;
+ *   - the model table, row "Weights": group size 128.
+ * Where the card is silent the reading taken is stated at the routine.
+ *
+ * Floating point: IEEE binary32 for the activation quantiser (the decision
+ * that produces an integer code is taken in fp32 on both sides), binary64
+ * for the layer output.  Build without -ffast-math and with
+ * -ffp-contract=off so that every operation is one correctly rounded IEEE
+ * operation.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_GROUP 128
+#define ORACLE_DRAFT 0
+#define ORACLE_TARGET 1
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ---- fp16 (IEEE binary16) decoding, from the format's definition ------- */
+/* 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.  Every binary16
+ * value is exactly representable in binary32 and binary64.              */
+double oracle_half_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int f = h & 0x3ff;
+  double v;
+  if (e == 0)
+    v = ldexp((double)f, -24); /* zero or subnormal: f * 2^-24 */
+  else if (e == 31)
+    v = f ? NAN : INFINITY;
+  else
+    v = ldexp((double)(1024 + f), e - 25); /* (1 + f/1024) * 2^(e-15) */
+  return sign ? -v : v;
+}
+
+float oracle_half_to_float(uint16_t h) { return (float)oracle_half_to_double(h); }
+
+/* ---- plane packing (model card, "Files": byte j = col 2j | col 2j+1 << 4) */
+void oracle_pack_plane(const uint8_t *u, int64_t N, int64_t K, uint8_t *plane) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < K / 2; ++j) {
+      uint8_t low = u[n * K + 2 * j] & 0xf;
+      uint8_t high = u[n * K + 2 * j + 1] & 0xf;
+      plane[n * (K / 2) + j] = (uint8_t)(low | (high << 4));
+    }
+}
+
+void oracle_unpack_plane(const uint8_t *plane, int64_t N, int64_t K, uint8_t *u) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      uint8_t byte = plane[n * (K / 2) + k / 2];
+      u[n * K + k] = (k % 2 == 0) ? (byte & 0xf) : (byte >> 4);
+    }
+}
+
+/* nibble of column k in row n of a plane */
+static int nibble(const uint8_t *plane, int64_t K, int64_t n, int64_t k) {
+  uint8_t byte = plane[n * (K / 2) + k / 2];
+  return (k % 2 == 0) ? (byte & 0xf) : (byte >> 4);
+}
+
+/* Integer weight code of the model card's formulas, before the scale:
+ *   draft  : hi - 8                      in [-8, 7]
+ *   target : 16 * (hi - 8) + (lo - 8)    in [-136, 119]
+ * (the target code does not fit int8; it is taken literally).           */
+static int weight_code(int mode, const uint8_t *hi, const uint8_t *lo, int64_t K,
+                       int64_t n, int64_t k) {
+  int h = nibble(hi, K, n, k);
+  if (mode == ORACLE_DRAFT) return h - 8;
+  int l = nibble(lo, K, n, k);
+  return 16 * (h - 8) + (l - 8);
+}
+
+/* ---- dequantised weights (model card, "Files", the two formulas) ------- */
+void oracle_dequant(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                    int64_t N, int64_t K, double *W) {
+  int64_t G = K / ORACLE_GROUP;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      double s = oracle_half_to_double(scale[n * G + k / ORACLE_GROUP]);
+      int h = nibble(hi, K, n, k);
+      if (mode == ORACLE_DRAFT) {
+        W[n * K + k] = (double)(h - 8) * s;
+      } else {
+        int l = nibble(lo, K, n, k);
+        W[n * K + k] = (double)(16 * (h - 8) + (l - 8)) * s / 16.0;
+      }
+    }
+}
+
+/* ---- symmetric int8 activation quantiser --------------------------------
+ * Model card, model table row "Activations": symmetric int8 per token, and
+ * per 128-column group for o_proj.  Readings where the card is silent:
+ *   scale s = max|x| / 127 in fp32 (one correctly rounded division);
+ *   q = round-half-even(x / s) (one correctly rounded fp32 division, then
+ *   rounding to the nearest integer, ties to even), clamped to [-127, 127];
+ *   a row (group) whose max|x| is 0 gets s = 0 and q = 0 (no division).
+ * group == 0: one scale per token, xs is [M];
+ * group == 128: one scale per (token, 128-column group), xs is [M, K/128]. */
+void oracle_quantize(const uint16_t *x, int64_t M, int64_t K, int group, int8_t *q,
+                     float *xs) {
+  int64_t span = (group == 0) ? K : group;
+  int64_t nspan = K / span;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t t = 0; t < nspan; ++t) {
+      const uint16_t *xr = x + m * K + t * span;
+      int8_t *qr = q + m * K + t * span;
+      float amax = 0.0f;
+      for (int64_t k = 0; k < span; ++k) {
+        float a = fabsf(oracle_half_to_float(xr[k]));
+        if (a > amax) amax = a;
+      }
+      float s = amax / 127.0f;
+      xs[m * nspan + t] = s;
+      for (int64_t k = 0; k < span; ++k) {
+        if (s == 0.0f) {
+          qr[k] = 0;
+          continue;
+        }
+        float ratio = oracle_half_to_float(xr[k]) / s;
+        float r = nearbyintf(ratio); /* default rounding: to nearest, ties to even */
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        qr[k] = (int8_t)r;
+      }
+    }
+}
+
+/* ---- per-group integer sums ----------------------------------------------
+ * S[m, n, g] = sum over the 128 columns k of group g of q[m, k] * code[n, k],
+ * with code the integer weight code above.  Summed in int64; returns the
+ * number of sums that do not fit int32 (always 0 for valid inputs).     */
+int64_t oracle_group_sums(int mode, const uint8_t *hi, const uint8_t *lo, const int8_t *q,
+                          int64_t M, int64_t N, int64_t K, int32_t *S) {
+  int64_t G = K / ORACLE_GROUP;
+  int64_t overflow = 0;
+#pragma omp parallel for reduction(+ : overflow) schedule(static)
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t m = 0; m < M; ++m)
+      for (int64_t g = 0; g < G; ++g) {
+        int64_t acc = 0;
+        for (int64_t k = g * ORACLE_GROUP; k < (g + 1) * ORACLE_GROUP; ++k)
+          acc += (int64_t)q[m * K + k] * weight_code(mode, hi, lo, K, n, k);
+        if (acc > INT32_MAX || acc < INT32_MIN) ++overflow;
+        S[(m * N + n) * G + g] = (int32_t)acc;
+      }
+  return overflow;
+}
+
+/* ---- the layer output -----------------------------------------------------
+ * y[m, n] = sum_k xdeq[m, k] * W[n, k] + bias[n], in fp64, with
+ *   xdeq[m, k] = q[m, k] * xs  (xs per token, or per (token, group))
+ *   W[n, k]    = the model card's draft or target dequantised weight.
+ * bias may be NULL.  The output rows n and tokens m computed are the lists
+ * rows[0..nrows) and toks[0..ntoks); y is [ntoks, nrows] (row-major).    */
+void oracle_linear_subset(int mode, const uint8_t *hi, const uint8_t *lo,
+                          const uint16_t *scale, const int8_t *q, const float *xs,
+                          int64_t M, int64_t N, int64_t K, int act_group,
+                          const uint16_t *bias, const int64_t *toks, int64_t ntoks,
+                          const int64_t *rows, int64_t nrows, double *y) {
+  int64_t G = K / ORACLE_GROUP;
+  (void)M;
+  (void)N;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < nrows; ++i) {
+    int64_t n = rows[i];
+    for (int64_t j = 0; j < ntoks; ++j) {
+      int64_t m = toks[j];
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        int64_t g = k / ORACLE_GROUP;
+        double xsv = (act_group == 0) ? (double)xs[m] : (double)xs[m * G + g];
+        double xdeq = (double)q[m * K + k] * xsv;
+        double s = oracle_half_to_double(scale[n * G + g]);
+        double w;
+        if (mode == ORACLE_DRAFT)
+          w = (double)(nibble(hi, K, n, k) - 8) * s;
+        else
+          w = (double)(16 * (nibble(hi, K, n, k) - 8) + (nibble(lo, K, n, k) - 8)) * s / 16.0;
+        acc += xdeq * w;
+      }
+      if (bias) acc += oracle_half_to_double(bias[n]);
+      y[j * nrows + i] = acc;
+    }
+  }
+}
+
+/* Full output y [M, N]. */
+void oracle_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                   const int8_t *q, const float *xs, int64_t M, int64_t N, int64_t K,
+                   int act_group, const uint16_t *bias, double *y) {
+  int64_t *toks = (int64_t *)malloc(sizeof(int64_t) * (size_t)(M > 0 ? M : 1));
+  int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)(N > 0 ? N : 1));
+  for (int64_t m = 0; m < M; ++m) toks[m] = m;
+  for (int64_t n = 0; n < N; ++n) rows[n] = n;
+  oracle_linear_subset(mode, hi, lo, scale, q, xs, M, N, K, act_group, bias, toks, M, rows,
+                       N, y);
+  free(toks);
+  free(rows);
+}
