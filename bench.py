@@ -1,0 +1,474 @@
+"""Benchmark of the BitNest nested W4/W8 linear layer on B200.
+
+One step = the decode hot path over the seven Llama-3-8B-shaped projections
+(q/o 4096x4096, k/v 1024x4096, gate/up 14336x4096, down 4096x14336, group
+128): for every projection the draft pass (activation quantise + W4A8 linear
+at M = 1, hi plane only) and the verify pass (quantise + W8A8 linear at
+M = 4 = gamma + 1, hi and lo planes); o_proj activations are quantised per
+128-group.  Inputs are seeded synthetic tensors of those shapes, resident in
+HBM.  The metric is HBM throughput: the algorithmic bytes the step must move
+(weights, scales, activations, outputs) divided by the device time.
+
+Also reported: the dominant kernel against the HBM roofline, an end-to-end
+number with host buffers (activation upload and output download inside the
+timed region), and the CPU oracle timed on a bounded sample of the same work.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w8_quantized_linear_b200 import synth  # noqa: E402
+
+METRIC = "HBM GB/s and % of 8 TB/s for draft/target GEMV; int8 TOPS % peak at prefill"
+UNIT = "GB/s"
+N_COPIES = 4  # rotating weight copies: 4 x 218 MB of planes, far above the 126 MB L2
+DECODE_M = {0: 1, 1: 4}  # draft at M = 1, target (verify) at M = gamma + 1 = 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def linear_bytes(mode, M, N, K):
+    """Algorithmic bytes of one linear launch: planes read once (hi, or hi and
+    lo), fp16 group scales, int8 activations and their fp32 scales, fp32 output."""
+    G = K // 128
+    planes = (1 if mode == 0 else 2) * N * K // 2
+    return planes + 2 * N * G + M * K + 4 * M + 4 * M * N
+
+
+def quant_bytes(M, K, act_group):
+    G = K // 128
+    return 2 * M * K + M * K + 4 * (M if act_group == 0 else M * G) + 4 * M * G
+
+
+class ClockSampler:
+    """NVML samples of SM clock and throttle reasons while the timed region runs."""
+
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index, period=0.02):
+        self.samples = []
+        self.reasons = set()
+        self.period = period
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = device_index
+            if vis:
+                ids = [v for v in vis.split(",") if v.strip()]
+                if device_index < len(ids) and ids[device_index].strip().isdigit():
+                    idx = int(ids[device_index])
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # no NVML: clocks are reported as unknown
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        return {
+            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+            "sm_max_mhz": self.max_mhz,
+            "reasons": sorted(self.reasons),
+            "samples": len(self.samples),
+        }
+
+
+def dominant_traffic(kernel_tag):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if that summary was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel_tag]
+        src = os.path.join(ROOT, rec["source"])
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if sha != rec["source_sha"]:
+            return None
+        return rec["bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- workload
+class DecodeWorkload:
+    """Weights (N_COPIES rotating copies), activations and outputs on one GPU."""
+
+    def __init__(self, device, n_copies=N_COPIES):
+        import torch
+
+        import w8_quantized_linear_b200 as bn
+
+        self.bn = bn
+        self.dev = device
+        self.projs = list(synth.LLAMA3_8B_PROJECTIONS.items())
+        self.copies = []  # per copy: {name: (hi, lo, scale)}
+        base = {}
+        for name, (N, K, _) in self.projs:
+            pid = synth.PROJ_IDS[name]
+            uh = torch.from_numpy(synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K))
+            ul = torch.from_numpy(synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K))
+            hi, lo = bn.pack_planes(uh.to(device), ul.to(device))
+            s = torch.from_numpy(synth.group_scales(synth.SEED_SCALES + pid, N, K)).to(device)
+            base[name] = (hi, lo, s)
+        self.copies.append(base)
+        for _ in range(1, n_copies):
+            self.copies.append({k: tuple(t.clone() for t in v) for k, v in base.items()})
+        # activations (fp16, device and pinned host) and the buffers of the step
+        self.x = {}
+        self.x_host = {}
+        self.bufs = {}
+        for name, (N, K, g) in self.projs:
+            pid = synth.PROJ_IDS[name]
+            for mode, M in DECODE_M.items():
+                xh = torch.from_numpy(synth.activations(synth.SEED_ACTS + pid + 100 * mode, M, K))
+                self.x_host[name, mode] = xh.pin_memory()
+                self.x[name, mode] = xh.to(device)
+                G = K // 128
+                self.bufs[name, mode] = dict(
+                    xq=torch.empty((M, K), dtype=torch.int8, device=device),
+                    xs=torch.empty((M,) if g == 0 else (M, G), dtype=torch.float32, device=device),
+                    xsum=torch.empty((M, G), dtype=torch.int32, device=device),
+                    y=torch.empty((M, N), dtype=torch.float32, device=device),
+                    y_host=torch.empty((M, N), dtype=torch.float32).pin_memory(),
+                )
+        torch.cuda.synchronize()
+
+    def step_bytes(self):
+        tot = 0
+        for name, (N, K, g) in self.projs:
+            for mode, M in DECODE_M.items():
+                tot += linear_bytes(mode, M, N, K) + quant_bytes(M, K, g)
+        return tot
+
+    def launches_per_step(self):
+        return 2 * 2 * len(self.projs)
+
+    def io_bytes(self):
+        h2d = sum(t.numel() * t.element_size() for t in self.x_host.values())
+        d2h = sum(b["y_host"].numel() * 4 for b in self.bufs.values())
+        return h2d, d2h
+
+    def run_step(self, copy, events=None, e2e=False):
+        """Enqueue one step on the current stream; `events`: per (name, mode)
+        (start, end) CUDA events recorded around each linear launch."""
+        bn = self.bn
+        w = self.copies[copy]
+        for mode in (0, 1):
+            for name, (N, K, g) in self.projs:
+                b = self.bufs[name, mode]
+                x = self.x[name, mode]
+                if e2e:
+                    x.copy_(self.x_host[name, mode], non_blocking=True)
+                bn.quantize_act(x, g, out=(b["xq"], b["xs"], b["xsum"]))
+                hi, lo, s = w[name]
+                if events is not None:
+                    events[name, mode][0].record()
+                bn.linear(mode, hi, lo, s, b["xq"], b["xs"], b["xsum"], g, out=b["y"])
+                if events is not None:
+                    events[name, mode][1].record()
+                if e2e:
+                    b["y_host"].copy_(b["y"], non_blocking=True)
+
+
+def capture(fn):
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm: first-launch host setup happens outside capture
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_replays(graphs, steps, barrier):
+    import torch
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    end.record()
+    torch.cuda.synchronize()
+    barrier()
+    return start.elapsed_time(end) / 1e3  # seconds
+
+
+# -------------------------------------------------------------- CPU oracle
+def cpu_baseline(rows_per_proj=256, budget_s=20.0):
+    """The oracle, as it stands, on the host cores: every projection and both
+    passes of the step on a sample of output rows, scaled to the whole step."""
+    import oracle
+
+    oracle.build()
+    t_total = 0.0
+    sampled = 0
+    for name, (N, K, g) in synth.LLAMA3_8B_PROJECTIONS.items():
+        pid = synth.PROJ_IDS[name]
+        rows = min(rows_per_proj, N)
+        uh = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K, 0, rows)
+        ul = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K, 0, rows)
+        s = synth.group_scales(synth.SEED_SCALES + pid, N, K, 0, rows)
+        hi, lo = oracle.pack_plane(uh), oracle.pack_plane(ul)
+        for mode, M in DECODE_M.items():
+            x = synth.activations(synth.SEED_ACTS + pid + 100 * mode, M, K)
+            t0 = time.perf_counter()
+            q, xs = oracle.quantize(x, g)
+            oracle.linear(mode, hi, lo if mode else None, s, q, xs, K, g)
+            dt = time.perf_counter() - t0
+            t_total += dt * (N / rows)  # scale the row sample to the full projection
+            sampled += rows
+    return t_total, oracle.num_threads(), sampled
+
+
+# ------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="bitnest", choices=["bitnest", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl_name = "llama3-8b-decode-projections"
+
+    if args.impl == "reference":
+        run_reference(args, rank, world, wl_name)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = DecodeWorkload(device)
+    step_bytes = wl.step_bytes()
+    graphs = [capture(lambda c=c: wl.run_step(c)) for c in range(N_COPIES)]
+    e2e_graphs = [capture(lambda c=c: wl.run_step(c, e2e=True)) for c in range(N_COPIES)]
+
+    for i in range(args.warmup):
+        graphs[i % N_COPIES].replay()
+    torch.cuda.synchronize()
+
+    with ClockSampler(local_rank) as clocks:
+        t = timed_replays(graphs, args.steps, barrier)
+    t = max_over_ranks(t)
+    ms_per_step = 1e3 * t / args.steps
+    value = world * step_bytes * args.steps / t / 1e9
+
+    # end to end: activations uploaded from pinned host memory and outputs read back
+    for i in range(args.warmup):
+        e2e_graphs[i % N_COPIES].replay()
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(timed_replays(e2e_graphs, args.steps, barrier))
+    e2e_value = world * step_bytes * args.steps / t_e2e / 1e9
+    h2d, d2h = wl.io_bytes()
+
+    # dominant kernel: the verify (target, M = 4) GEMV.  Per-launch device
+    # time from CUDA events recorded on the launching stream right around each
+    # launch; a spin kernel first lets the host enqueue the whole sequence, so
+    # no launch waits on the host between its two events.
+    events = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for k in wl.bufs}
+    dur = {k: 0.0 for k in events}
+    n_ev = max(8, min(args.steps, 200))
+    for i in range(n_ev):
+        torch.cuda._sleep(400_000)
+        wl.run_step(i % N_COPIES, events=events)
+        torch.cuda.synchronize()
+        for k, (a, b) in events.items():
+            dur[k] += a.elapsed_time(b) / 1e3
+    target_keys = [k for k in events if k[1] == 1]
+    draft_keys = [k for k in events if k[1] == 0]
+    tgt_bytes = sum(linear_bytes(1, 4, *synth.LLAMA3_8B_PROJECTIONS[k[0]][:2]) for k in target_keys)
+    tgt_time = sum(dur[k] for k in target_keys) / n_ev
+    drf_bytes = sum(linear_bytes(0, 1, *synth.LLAMA3_8B_PROJECTIONS[k[0]][:2]) for k in draft_keys)
+    drf_time = sum(dur[k] for k in draft_keys) / n_ev
+    hbm_peak, bf16_peak, peak_kind = load_peaks()
+    per_proj = {}
+    for (name, mode) in events:
+        N, K, _ = synth.LLAMA3_8B_PROJECTIONS[name]
+        d = dur[name, mode] / n_ev
+        b = linear_bytes(mode, DECODE_M[mode], N, K)
+        per_proj[f"{name}/{'draft' if mode == 0 else 'target'}"] = {
+            "us": round(d * 1e6, 3), "GB/s": round(b / d / 1e9, 1),
+            "frac_hbm": round(b / d / 1e9 / hbm_peak, 3)}
+    achieved = tgt_bytes / tgt_time / 1e9
+    roofline = {
+        "bound": "hbm",
+        "kernel": "gemv_kernel<TARGET, M=4> (7 projections)",
+        "achieved": round(achieved, 1),
+        "peak": hbm_peak,
+        "unit": "GB/s",
+        "frac": round(achieved / hbm_peak, 4),
+        "peak_kind": f"{peak_kind} (copy bandwidth)",
+        "traffic": dominant_traffic("gemv_target_m4"),
+        "algorithmic_bytes_per_launch": round(tgt_bytes / len(target_keys)),
+        "draft_gemv_achieved": round(drf_bytes / drf_time / 1e9, 1),
+        "draft_gemv_frac": round(drf_bytes / drf_time / 1e9 / hbm_peak, 4),
+        "per_projection": per_proj,
+    }
+    for g in graphs + e2e_graphs:
+        g.reset()
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8 x u8/u4 -> int32, fp32 epilogue",
+        "data": "synthetic (seeded SplitMix64: uniform nibbles, fp16 scales, N(0,1) activations with 4 x20 outliers)",
+        "config": {
+            "workload": wl_name,
+            "projections": {k: list(v[:2]) for k, v in synth.LLAMA3_8B_PROJECTIONS.items()},
+            "passes": "draft W4A8 M=1 + target W8A8 M=4 per projection, quantise included",
+            "group": 128,
+            "bytes_per_step": step_bytes,
+            "l2": f"inputs larger than L2: {N_COPIES} rotating weight copies "
+                  f"({N_COPIES * sum(v[0] * v[1] for v in synth.LLAMA3_8B_PROJECTIONS.values()) / 1e6:.0f} MB of planes)",
+            "parallelism": "replicas" if world > 1 else "single",
+            "timing": "CUDA graph per step, CUDA events on the launching stream",
+        },
+        "clocks": clocks.summary(),
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "activations uploaded from pinned host memory and outputs read back every step; weights resident"},
+        "gpu_launches": wl.launches_per_step() * args.steps,
+        "roofline": roofline,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_cpu, cores, rows = cpu_baseline()
+        out["cpu_baseline"] = {
+            "value": round(step_bytes / t_cpu / 1e9, 4), "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"every projection, both passes, first {rows // 14} output rows each "
+                      f"({rows} row-passes), time scaled by N/rows to one full step",
+        }
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_reference(args, rank, world, wl_name):
+    """The oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    step_bytes = 0
+    for name, (N, K, g) in synth.LLAMA3_8B_PROJECTIONS.items():
+        for mode, M in DECODE_M.items():
+            step_bytes += linear_bytes(mode, M, N, K) + quant_bytes(M, K, g)
+    rows = 64
+    for _ in range(min(args.warmup, 1)):
+        cpu_baseline(rows_per_proj=rows)
+    times = []
+    for _ in range(args.steps if args.steps <= 5 else 5):
+        t, cores, sampled = cpu_baseline(rows_per_proj=rows)
+        times.append(t)
+    t = statistics.median(times)
+    value = step_bytes / t / 1e9
+    out = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": len(times), "warmup": args.warmup, "ms_per_step": round(1e3 * t, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int64 sums, fp64 output", "data": "synthetic",
+        "config": {"workload": wl_name},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"first {rows} output rows of every projection and pass, "
+                                   "scaled by N/rows to one full step"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

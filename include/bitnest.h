@@ -1,0 +1,159 @@
+/*
+ * bitnest.h -- C ABI of the BitNest bit-nested W4/W8 quantised linear layer
+ * on NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (BitNest-Llama-3-8B model card, section "Files",
+ * planes.safetensors entry, and the model table rows "Weights" and
+ * "Activations"): one stored 8-bit weight code serves two precisions.
+ *   hi, lo : uint8 [N, K/2] planes of unsigned nibbles u = q + 8; byte j of a
+ *            row holds column 2j in its low nibble and column 2j+1 in its high
+ *            nibble.
+ *   scale  : fp16 [N, K/128], one scale per 128-column group.
+ *   draft  (W4A8) reads hi only:   W4[n,k] = (hi - 8) * scale
+ *   target (W8A8) reads hi and lo: W8[n,k] = (16*(hi - 8) + (lo - 8)) * scale / 16
+ *   activations are symmetric int8, one scale per token (per 128-column
+ *   group for o_proj): x[m,k] ~= xq[m,k] * xscale.
+ *   y[m,n] = sum_k (xq[m,k] * xscale) * W[n,k] (+ bias[n]).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers to row-major, contiguous
+ *     arrays; the caller allocates, owns and frees them.  The library
+ *     allocates no memory and keeps no state beyond cached device
+ *     attributes and driver entry points.
+ *   - fp16 arrays are passed as their IEEE binary16 bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously on it; the entry points are re-entrant.
+ *   - Every argument check runs on the host, before anything is launched.  A
+ *     failed check returns a non-zero BITNEST_ERR_* status and launches
+ *     nothing.  A launch failure returns BITNEST_ERR_CUDA.  Faults during
+ *     execution surface at the caller's next synchronisation.
+ *   - M == 0 or N == 0 is an empty problem: BITNEST_OK, nothing launched, and
+ *     the pointers are not inspected (after mode / group / K are checked).
+ *   - K must be a positive multiple of 128 (the group size).
+ *   - Base pointers must be 16-byte aligned (BITNEST_ERR_MISALIGNED).
+ */
+#ifndef BITNEST_H_
+#define BITNEST_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Which model reads the planes. */
+#define BITNEST_DRAFT 0  /* W4A8: hi plane only        */
+#define BITNEST_TARGET 1 /* W8A8: hi and lo planes    */
+
+/* Kernel family for bitnest_linear_path. */
+#define BITNEST_PATH_AUTO 0 /* the library picks (see bitnest_select_path)          */
+#define BITNEST_PATH_GEMV 1 /* CUDA-core decode GEMV: dp4a, M <= BITNEST_GEMV_MAX_M  */
+#define BITNEST_PATH_TC 2   /* tcgen05 kind::i8 tensor-core GEMM, any M              */
+
+#define BITNEST_GEMV_MAX_M 8 /* largest M the GEMV kernels are built for */
+
+/* Status codes. */
+#define BITNEST_OK 0
+#define BITNEST_ERR_INVALID_ARG 1       /* null pointer, bad mode / group / path        */
+#define BITNEST_ERR_UNSUPPORTED_SHAPE 2 /* K not a positive multiple of 128, sizes < 0 */
+#define BITNEST_ERR_MISALIGNED 3        /* a base pointer is not 16-byte aligned       */
+#define BITNEST_ERR_CUDA 4              /* a CUDA launch or driver call failed         */
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *bitnest_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int bitnest_version(void);
+
+/* Every wait of the tensor-core kernels on another warp or on a copy is
+ * bounded; a wait that gives up sets a device flag and the kernel winds down
+ * without finishing its output.  Returns that flag for the current device (1:
+ * some launch since the last reset gave up, its outputs are invalid; 0: none),
+ * or -BITNEST_ERR_CUDA.  Synchronous: reads device memory.  reset != 0 clears
+ * the flag after reading it. */
+int bitnest_device_wait_timeout(int reset);
+
+/*
+ * Pack unpacked nibbles into the planes of the model card's layout
+ * ("Files": byte j holds column 2j in its low nibble, 2j+1 in its high).
+ *   uh, ul : uint8 [N, K] nibble values; only the low 4 bits are used.
+ *            ul may be NULL (then lo is not written; lo may be NULL too).
+ *   hi, lo : uint8 [N, K/2] outputs.
+ * K must be a positive multiple of 128.
+ */
+int bitnest_pack_planes(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K,
+                        uint8_t *hi, uint8_t *lo, void *stream);
+
+/*
+ * Symmetric int8 activation quantiser (model table row "Activations").
+ *   x         : fp16 [M, K] activations (finite values).
+ *   act_group : 0   -> one scale per token;   xscale is fp32 [M]
+ *               128 -> one scale per (token, 128-column group) (o_proj);
+ *                      xscale is fp32 [M, K/128].
+ *   xq        : int8 [M, K] output, q = clamp(rne(x / s), -127, 127) with
+ *               s = max|x| / 127 computed in fp32 (correctly rounded
+ *               division, round-half-even); an all-zero span gives s = 0, q = 0.
+ *   xsum      : int32 [M, K/128] output, xsum[m,g] = sum of xq[m,k] over the
+ *               128 columns of group g; may be NULL (not written).
+ *               bitnest_linear needs it (see there).
+ */
+int bitnest_quantize_act(const uint16_t *x, int64_t M, int64_t K, int act_group, int8_t *xq,
+                         float *xscale, int32_t *xsum, void *stream);
+
+/*
+ * Per-128-group sums of already quantised activations:
+ *   xsum[m, g] = sum_{k in group g} xq[m, k]   (int32 [M, K/128]).
+ * For callers whose xq does not come from bitnest_quantize_act.
+ */
+int bitnest_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
+                           void *stream);
+
+/*
+ * The nested linear layer, y = dequant(xq, xscale) * W^T (+ bias), with W the
+ * draft (mode = BITNEST_DRAFT, W4A8) or target (BITNEST_TARGET, W8A8) weight.
+ *   hi, lo    : uint8 [N, K/2] planes; lo is ignored (may be NULL) for DRAFT
+ *               and required for TARGET.
+ *   scale     : fp16 [N, K/128] group scales.
+ *   xq        : int8 [M, K] quantised activations.
+ *   xscale    : fp32 [M] (act_group 0) or [M, K/128] (act_group 128).
+ *   xsum      : int32 [M, K/128] group sums of xq (bitnest_quantize_act
+ *               writes them).  Required: the tensor-core path folds the
+ *               planes' unsigned-nibble offset (8 for hi, 136 for the
+ *               combined byte) into one correction per (token, group) and
+ *               takes it from here; it must match xq.
+ *   y         : fp32 [M, N] output.
+ *   bias      : fp16 [N] or NULL.
+ * Integer group sums are exact (int32); the epilogue is fp32, so y agrees
+ * with an exact evaluation to within fp32 summation rounding.
+ */
+int bitnest_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                   const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
+                   int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
+                   void *stream);
+
+/* bitnest_linear with an explicit kernel family (BITNEST_PATH_*).  PATH_GEMV
+ * requires M <= BITNEST_GEMV_MAX_M (else BITNEST_ERR_UNSUPPORTED_SHAPE). */
+int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                        const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
+                        int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
+                        int path, void *stream);
+
+/* The kernel family BITNEST_PATH_AUTO picks for this problem (host only,
+ * launches nothing).  Returns BITNEST_PATH_GEMV or BITNEST_PATH_TC. */
+int bitnest_select_path(int mode, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Test hook: the exact int32 group sums the kernels of `path` form,
+ *   S[m, n, g] = sum_{k in g} xq[m,k] * code[n,k],
+ * code = hi - 8 (DRAFT) or 16*(hi - 8) + (lo - 8) (TARGET), written to
+ * S int32 [M, N, K/128].  Same inner loops as bitnest_linear_path.
+ */
+int bitnest_debug_group_sums(int mode, const uint8_t *hi, const uint8_t *lo,
+                             const int8_t *xq, const int32_t *xsum, int64_t M, int64_t N,
+                             int64_t K, int32_t *S, int path, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNEST_H_ */

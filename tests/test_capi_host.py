@@ -1,0 +1,118 @@
+"""The C ABI library on the host (no GPU): it loads, exports every symbol the
+header declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w8_quantized_linear_b200 as bn
+from w8_quantized_linear_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitnest.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return bn.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitnest_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("bitnest_pack_planes", "bitnest_quantize_act", "bitnest_linear",
+                     "bitnest_debug_group_sums", "bitnest_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_status_strings(L):
+    assert bn.status_string(0) == "ok"
+    for s in range(1, 5):
+        assert bn.status_string(s) not in ("ok", "unknown status")
+    assert bn.status_string(99) == "unknown status"
+    assert L.bitnest_version() >= 100
+
+
+def test_select_path():
+    assert bn.select_path(bn.DRAFT, 1, 4096, 4096) == bn.PATH_GEMV
+    assert bn.select_path(bn.TARGET, 4, 14336, 4096) == bn.PATH_GEMV
+    assert bn.select_path(bn.TARGET, 8, 4096, 14336) == bn.PATH_GEMV
+    assert bn.select_path(bn.TARGET, 9, 4096, 4096) == bn.PATH_TC
+    assert bn.select_path(bn.TARGET, 2048, 4096, 4096) == bn.PATH_TC
+
+
+A = 0x10000  # fake, aligned, never dereferenced (every call below fails before a launch)
+MIS = 0x10001
+
+
+def _lin(L, mode=1, hi=A, lo=A, scale=A, xq=A, xs=A, xsum=A, M=4, N=64, K=128, y=A, g=0,
+         bias=None, path=0):
+    v = ctypes.c_void_p
+    return L.bitnest_linear_path(mode, v(hi), v(lo), v(scale), v(xq), v(xs), v(xsum), M, N, K,
+                                 v(y), g, v(bias) if bias else None, path, None)
+
+
+def test_linear_argument_checks(L):
+    assert _lin(L, mode=2) == 1
+    assert _lin(L, g=64) == 1
+    assert _lin(L, path=3) == 1
+    assert _lin(L, K=0) == 2
+    assert _lin(L, K=100) == 2
+    assert _lin(L, K=4096 + 64) == 2
+    assert _lin(L, M=-1) == 2
+    assert _lin(L, hi=0) == 1
+    assert _lin(L, scale=0) == 1
+    assert _lin(L, xsum=0) == 1
+    assert _lin(L, y=0) == 1
+    assert _lin(L, mode=1, lo=0) == 1
+    assert _lin(L, mode=1, lo=MIS) == 3
+    assert _lin(L, hi=MIS) == 3
+    assert _lin(L, y=MIS) == 3
+    assert _lin(L, bias=MIS) == 3
+    # draft ignores lo entirely (NULL or misaligned)
+    assert _lin(L, mode=0, lo=0, M=0) == 0
+    assert _lin(L, mode=0, lo=MIS, M=0) == 0
+    # empty problems launch nothing and succeed
+    assert _lin(L, M=0) == 0
+    assert _lin(L, N=0) == 0
+    # an explicit GEMV path cannot take more than 8 tokens (checked before launch)
+    assert _lin(L, M=9, path=1) == 2
+    assert L.bitnest_device_wait_timeout is not None
+
+
+def test_quantize_pack_sum_argument_checks(L):
+    v = ctypes.c_void_p
+    assert L.bitnest_quantize_act(v(A), 4, 128, 3, v(A), v(A), None, None) == 1
+    assert L.bitnest_quantize_act(v(A), 4, 130, 0, v(A), v(A), None, None) == 2
+    assert L.bitnest_quantize_act(None, 4, 128, 0, v(A), v(A), None, None) == 1
+    assert L.bitnest_quantize_act(v(A), 4, 128, 0, v(MIS), v(A), None, None) == 3
+    assert L.bitnest_quantize_act(v(A), 4, 128, 0, v(A), v(A), v(MIS), None) == 3
+    assert L.bitnest_quantize_act(v(A), 0, 128, 0, v(A), v(A), None, None) == 0
+    assert L.bitnest_pack_planes(v(A), None, 4, 127, v(A), None, None) == 2
+    assert L.bitnest_pack_planes(None, None, 4, 128, v(A), None, None) == 1
+    assert L.bitnest_pack_planes(v(A), v(A), 4, 128, v(A), None, None) == 1
+    assert L.bitnest_pack_planes(v(A), None, 0, 128, v(A), None, None) == 0
+    assert L.bitnest_act_group_sums(v(A), 4, 256, None, None) == 1
+    assert L.bitnest_act_group_sums(v(A), 0, 256, v(A), None) == 0
+    assert L.bitnest_debug_group_sums(1, v(A), None, v(A), v(A), 1, 1, 128, v(A), 0, None) == 1
+    assert L.bitnest_debug_group_sums(0, v(A), None, v(A), v(A), 0, 1, 128, v(A), 0, None) == 0
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(bn, "_lib", None)
+    monkeypatch.setattr(bn, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        bn.lib()

@@ -1,0 +1,109 @@
+"""GPU parity of the tcgen05 tensor-core path against the CPU oracle.
+
+Same bar as the decode GEMV: the int32 per-group sums equal the oracle's
+bit for bit; y satisfies max|y - y_ref| / (|y_ref| + 1e-3 rms(y_ref)) <= 1e-3.
+Shapes span several 128-row weight tiles and token tiles with ragged tails
+in both, and the Llama-3-8B-shaped prefill (M = 2048) on sampled outputs.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import w8_quantized_linear_b200 as bn
+from w8_quantized_linear_b200 import synth
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-3
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from test_gpu_parity import Problem, dev, host  # noqa: E402
+
+
+@pytest.fixture(autouse=True)
+def _no_wait_timeouts():
+    bn.device_wait_timeout(reset=True)
+    yield
+    torch.cuda.synchronize()
+    assert bn.device_wait_timeout(reset=True) == 0
+
+
+SHAPES = [(1, 1, 128), (9, 100, 256), (16, 128, 1024), (17, 129, 384), (33, 300, 1152),
+          (64, 256, 512), (100, 200, 4096), (128, 128, 128), (129, 257, 1024),
+          (300, 130, 640)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("mode", [0, 1])
+def test_tc_group_sums_bit_exact(M, N, K, mode):
+    p = Problem(M, N, K, seed=M + 3 * N)
+    S = bn.debug_group_sums(mode, p.d_hi, p.d_lo, p.d_xq, p.d_xsum, path=bn.PATH_TC)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(S), oracle.group_sums(mode, p.hi, p.lo, p.q, K))
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("act_group", [0, 128])
+def test_tc_output(M, N, K, mode, act_group):
+    p = Problem(M, N, K, seed=N + K + M, act_group=act_group)
+    y = p.y_gpu(mode, path=bn.PATH_TC)
+    assert oracle.max_normalised_error(y, p.y_ref(mode)) <= TOL
+
+
+def test_tc_bias():
+    p = Problem(20, 150, 512, seed=4, bias=True)
+    for mode in (0, 1):
+        assert oracle.max_normalised_error(p.y_gpu(mode, bn.PATH_TC), p.y_ref(mode)) <= TOL
+
+
+@pytest.mark.parametrize("M", [5, 40, 128])
+def test_tc_draft_equals_target_when_lo_is_eight(M):
+    p = Problem(M, 257, 1024, seed=6, lo_eight=True)
+    assert np.array_equal(p.y_gpu(0, bn.PATH_TC), p.y_gpu(1, bn.PATH_TC))
+
+
+@pytest.mark.parametrize("M", [1, 4, 8])
+def test_tc_and_gemv_agree(M):
+    p = Problem(M, 384, 2048, seed=11)
+    for mode in (0, 1):
+        y_tc = p.y_gpu(mode, bn.PATH_TC)
+        y_gv = p.y_gpu(mode, bn.PATH_GEMV)
+        ref = p.y_ref(mode)
+        assert oracle.max_normalised_error(y_tc, ref) <= TOL
+        assert oracle.max_normalised_error(y_gv, ref) <= TOL
+        S_tc = bn.debug_group_sums(mode, p.d_hi, p.d_lo, p.d_xq, p.d_xsum, path=bn.PATH_TC)
+        S_gv = bn.debug_group_sums(mode, p.d_hi, p.d_lo, p.d_xq, p.d_xsum, path=bn.PATH_GEMV)
+        assert torch.equal(S_tc, S_gv)
+
+
+@pytest.mark.parametrize("name", list(synth.LLAMA3_8B_PROJECTIONS))
+def test_llama3_prefill_sampled(name):
+    """Target W8A8 at M = 2048 on the full Llama-3-8B-shaped projection; the
+    oracle evaluates a sample of rows x tokens and the exact sums of a sample."""
+    N, K, act_group = synth.LLAMA3_8B_PROJECTIONS[name]
+    M = 2048
+    pid = synth.PROJ_IDS[name]
+    uh = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K)
+    ul = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K)
+    s = synth.group_scales(synth.SEED_SCALES + pid, N, K)
+    x = synth.activations(synth.SEED_ACTS + pid, M, K)
+    d_hi, d_lo = bn.pack_planes(dev(uh), dev(ul))
+    d_xq, d_xs, d_xsum = bn.quantize_act(dev(x), act_group)
+    y = host(bn.linear(1, d_hi, d_lo, dev(s), d_xq, d_xs, d_xsum, act_group))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(pid)
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.choice(N, 60, replace=False)]))
+    toks = np.unique(np.concatenate([[0, 127, 128, M - 1], rng.choice(M, 28, replace=False)]))
+    hi_r, lo_r = oracle.pack_plane(uh[rows]), oracle.pack_plane(ul[rows])
+    q, xs = oracle.quantize(x, act_group)
+    y_ref = oracle.linear(1, hi_r, lo_r, s[rows], q[toks], xs[toks], K, act_group)
+    assert oracle.max_normalised_error(y[np.ix_(toks, rows)], y_ref) <= TOL
+    # the exact int32 sums of a few weight tiles
+    S = bn.debug_group_sums(1, d_hi[:256], d_lo[:256], d_xq, d_xsum)
+    S = host(S)
+    S_ref = oracle.group_sums(1, oracle.pack_plane(uh[:256]), oracle.pack_plane(ul[:256]),
+                              q[toks], K)
+    assert np.array_equal(S[toks], S_ref)

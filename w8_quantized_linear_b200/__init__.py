@@ -1,0 +1,166 @@
+"""BitNest bit-nested W4/W8 quantised linear layer on B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libbitnest.so`` (declared in
+``include/bitnest.h``).  Every function here only marshals arguments: it
+allocates outputs with torch, passes device pointers and the current CUDA
+stream, and raises on a non-zero status.  All computation runs in the CUDA
+kernels of the library; there is no CPU path.  If the library is missing the
+first call raises.
+
+One stored 8-bit weight code serves two models (BitNest-Llama-3-8B model
+card, section "Files"): the draft (W4A8) reads the hi nibble plane only, the
+target (W8A8) reads the hi and lo planes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+DRAFT = 0
+TARGET = 1
+PATH_AUTO = 0
+PATH_GEMV = 1
+PATH_TC = 2
+GEMV_MAX_M = 8
+GROUP = 128
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitnest.so")
+
+_lib = None
+
+
+class BitnestError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbitnest.so (built in-tree by build.py); raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m w8_quantized_linear_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    L.bitnest_status_string.argtypes = [I]
+    L.bitnest_status_string.restype = ctypes.c_char_p
+    L.bitnest_version.restype = I
+    L.bitnest_device_wait_timeout.argtypes = [I]
+    L.bitnest_device_wait_timeout.restype = I
+    L.bitnest_pack_planes.argtypes = [P, P, I64, I64, P, P, P]
+    L.bitnest_quantize_act.argtypes = [P, I64, I64, I, P, P, P, P]
+    L.bitnest_act_group_sums.argtypes = [P, I64, I64, P, P]
+    L.bitnest_linear.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, P]
+    L.bitnest_linear_path.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, I, P]
+    L.bitnest_select_path.argtypes = [I, I64, I64, I64]
+    L.bitnest_debug_group_sums.argtypes = [I, P, P, P, P, I64, I64, I64, P, I, P]
+    for name in ("bitnest_pack_planes", "bitnest_quantize_act", "bitnest_act_group_sums",
+                 "bitnest_linear", "bitnest_linear_path", "bitnest_select_path",
+                 "bitnest_debug_group_sums"):
+        getattr(L, name).restype = I
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().bitnest_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise BitnestError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t=None):
+    import torch
+
+    dev = t.device if t is not None else None
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def device_wait_timeout(reset: bool = False) -> int:
+    """1 if a bounded in-kernel wait gave up since the last reset, else 0."""
+    v = int(lib().bitnest_device_wait_timeout(1 if reset else 0))
+    if v < 0:
+        raise BitnestError(-v, "bitnest_device_wait_timeout")
+    return v
+
+
+def select_path(mode: int, M: int, N: int, K: int) -> int:
+    return int(lib().bitnest_select_path(int(mode), int(M), int(N), int(K)))
+
+
+def pack_planes(uh, ul=None):
+    """uint8 nibbles [N, K] (and optionally ul) -> planes uint8 [N, K/2]."""
+    import torch
+
+    N, K = uh.shape
+    hi = torch.empty((N, K // 2), dtype=torch.uint8, device=uh.device)
+    lo = torch.empty_like(hi) if ul is not None else None
+    _check(lib().bitnest_pack_planes(_ptr(uh), _ptr(ul), N, K, _ptr(hi), _ptr(lo), _stream(uh)),
+           "bitnest_pack_planes")
+    return hi, lo
+
+
+def quantize_act(x, act_group: int = 0, with_sum: bool = True, out=None):
+    """fp16 [M, K] -> (xq int8 [M, K], xscale fp32 [M] or [M, K/128], xsum int32 [M, K/128])."""
+    import torch
+
+    M, K = x.shape
+    if out is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+        xs = torch.empty((M,) if act_group == 0 else (M, K // GROUP), dtype=torch.float32,
+                         device=x.device)
+        xsum = torch.empty((M, K // GROUP), dtype=torch.int32, device=x.device) if with_sum else None
+    else:
+        xq, xs, xsum = out
+    _check(lib().bitnest_quantize_act(_ptr(x), M, K, int(act_group), _ptr(xq), _ptr(xs),
+                                      _ptr(xsum), _stream(x)), "bitnest_quantize_act")
+    return xq, xs, xsum
+
+
+def act_group_sums(xq, out=None):
+    import torch
+
+    M, K = xq.shape
+    xsum = out if out is not None else torch.empty((M, K // GROUP), dtype=torch.int32,
+                                                    device=xq.device)
+    _check(lib().bitnest_act_group_sums(_ptr(xq), M, K, _ptr(xsum), _stream(xq)),
+           "bitnest_act_group_sums")
+    return xsum
+
+
+def linear(mode: int, hi, lo, scale, xq, xscale, xsum, act_group: int = 0, bias=None,
+           out=None, path: int = PATH_AUTO):
+    """The nested linear layer: fp32 y [M, N]."""
+    import torch
+
+    M, K = xq.shape
+    N = hi.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=xq.device)
+    _check(lib().bitnest_linear_path(int(mode), _ptr(hi), _ptr(lo), _ptr(scale), _ptr(xq),
+                                     _ptr(xscale), _ptr(xsum), M, N, K, _ptr(y), int(act_group),
+                                     _ptr(bias), int(path), _stream(xq)), "bitnest_linear")
+    return y
+
+
+def debug_group_sums(mode: int, hi, lo, xq, xsum, path: int = PATH_AUTO, out=None):
+    """int32 [M, N, K/128] exact group sums, from the same inner loops as `linear`."""
+    import torch
+
+    M, K = xq.shape
+    N = hi.shape[0]
+    S = out if out is not None else torch.empty((M, N, K // GROUP), dtype=torch.int32,
+                                                 device=xq.device)
+    _check(lib().bitnest_debug_group_sums(int(mode), _ptr(hi), _ptr(lo), _ptr(xq), _ptr(xsum),
+                                          M, N, K, _ptr(S), int(path), _stream(xq)),
+           "bitnest_debug_group_sums")
+    return S

@@ -1,0 +1,167 @@
+// C ABI of the BitNest nested W4/W8 linear layer: host-side argument checks
+// and dispatch to the sm_100a kernels.  Declarations and the contract of each
+// entry point are in include/bitnest.h.
+#include <stdint.h>
+
+#include "bitnest.h"
+#include "common.cuh"
+#include "launch.h"
+
+using namespace bitnest;
+
+namespace {
+
+bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? BITNEST_OK : BITNEST_ERR_CUDA; }
+
+// K must be a positive multiple of the group size; M, N non-negative.
+int check_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K <= 0 || K % kGroup != 0) return BITNEST_ERR_UNSUPPORTED_SHAPE;
+  // 32-bit grid / index limits of the kernels
+  if (K > (int64_t)1 << 24 || N > (int64_t)1 << 31 || M > (int64_t)1 << 31)
+    return BITNEST_ERR_UNSUPPORTED_SHAPE;
+  return BITNEST_OK;
+}
+
+int check_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                 const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
+                 int64_t N, int64_t K, const float *y, int act_group, const uint16_t *bias) {
+  if (mode != BITNEST_DRAFT && mode != BITNEST_TARGET) return BITNEST_ERR_INVALID_ARG;
+  if (act_group != 0 && act_group != kGroup) return BITNEST_ERR_INVALID_ARG;
+  int s = check_shape(M, N, K);
+  if (s != BITNEST_OK) return s;
+  if (M == 0 || N == 0) return BITNEST_OK;  // empty problem: pointers are not inspected
+  if (!hi || !scale || !xq || !xscale || !xsum || !y) return BITNEST_ERR_INVALID_ARG;
+  if (mode == BITNEST_TARGET && !lo) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(hi) || misaligned(scale) || misaligned(xq) || misaligned(xscale) ||
+      misaligned(xsum) || misaligned(y) || (bias && misaligned(bias)) ||
+      (mode == BITNEST_TARGET && misaligned(lo)))
+    return BITNEST_ERR_MISALIGNED;
+  return BITNEST_OK;
+}
+
+int pick_path(int mode, int64_t M, int64_t N, int64_t K) {
+  (void)mode;
+  (void)N;
+  if (gemv_fits(M, K)) return BITNEST_PATH_GEMV;
+  return BITNEST_PATH_TC;
+}
+
+int run_linear(const LinearArgs &a, int path, cudaStream_t st) {
+  if (path == BITNEST_PATH_AUTO) path = pick_path(a.mode, a.M, a.N, a.K);
+  if (path == BITNEST_PATH_GEMV) {
+    if (!gemv_fits(a.M, a.K)) return BITNEST_ERR_UNSUPPORTED_SHAPE;
+    return cuda_status(launch_gemv(a, st));
+  }
+  if (path == BITNEST_PATH_TC) {
+    if (!tc_supported(a.M, a.N, a.K)) return BITNEST_ERR_UNSUPPORTED_SHAPE;
+    return cuda_status(launch_tc(a, st));
+  }
+  return BITNEST_ERR_INVALID_ARG;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *bitnest_status_string(int status) {
+  switch (status) {
+    case BITNEST_OK: return "ok";
+    case BITNEST_ERR_INVALID_ARG: return "invalid argument";
+    case BITNEST_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case BITNEST_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case BITNEST_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+int bitnest_version(void) { return 100; }
+
+int bitnest_device_wait_timeout(int reset) {
+  int flag = 0;
+  if (read_wait_timeout(&flag, reset != 0) != cudaSuccess) return -BITNEST_ERR_CUDA;
+  return flag;
+}
+
+int bitnest_pack_planes(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K,
+                        uint8_t *hi, uint8_t *lo, void *stream) {
+  int s = check_shape(0, N, K);
+  if (s != BITNEST_OK) return s;
+  if (N == 0) return BITNEST_OK;
+  if (!uh || !hi || (ul && !lo)) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(uh) || misaligned(hi) || (ul && (misaligned(ul) || misaligned(lo))))
+    return BITNEST_ERR_MISALIGNED;
+  if (N == 0) return BITNEST_OK;
+  return cuda_status(launch_pack(uh, ul, N, K, hi, lo, (cudaStream_t)stream));
+}
+
+int bitnest_quantize_act(const uint16_t *x, int64_t M, int64_t K, int act_group, int8_t *xq,
+                         float *xscale, int32_t *xsum, void *stream) {
+  if (act_group != 0 && act_group != kGroup) return BITNEST_ERR_INVALID_ARG;
+  int s = check_shape(M, 0, K);
+  if (s != BITNEST_OK) return s;
+  if (M == 0) return BITNEST_OK;
+  if (!x || !xq || !xscale) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(x) || misaligned(xq) || misaligned(xscale) || (xsum && misaligned(xsum)))
+    return BITNEST_ERR_MISALIGNED;
+  if (M == 0) return BITNEST_OK;
+  return cuda_status(launch_quantize(x, M, K, act_group, xq, xscale, xsum, (cudaStream_t)stream));
+}
+
+int bitnest_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
+                           void *stream) {
+  int s = check_shape(M, 0, K);
+  if (s != BITNEST_OK) return s;
+  if (M == 0) return BITNEST_OK;
+  if (!xq || !xsum) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(xq) || misaligned(xsum)) return BITNEST_ERR_MISALIGNED;
+  if (M == 0) return BITNEST_OK;
+  return cuda_status(launch_act_group_sums(xq, M, K, xsum, (cudaStream_t)stream));
+}
+
+int bitnest_select_path(int mode, int64_t M, int64_t N, int64_t K) {
+  return pick_path(mode, M, N, K);
+}
+
+int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                        const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
+                        int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
+                        int path, void *stream) {
+  if (path < BITNEST_PATH_AUTO || path > BITNEST_PATH_TC) return BITNEST_ERR_INVALID_ARG;
+  int s = check_linear(mode, hi, lo, scale, xq, xscale, xsum, M, N, K, y, act_group, bias);
+  if (s != BITNEST_OK) return s;
+  if (M == 0 || N == 0) return BITNEST_OK;
+  LinearArgs a{mode, hi, mode == BITNEST_TARGET ? lo : nullptr, scale, xq, xscale, xsum,
+               bias, y, nullptr, M, N, K, act_group};
+  return run_linear(a, path, (cudaStream_t)stream);
+}
+
+int bitnest_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                   const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
+                   int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
+                   void *stream) {
+  return bitnest_linear_path(mode, hi, lo, scale, xq, xscale, xsum, M, N, K, y, act_group,
+                             bias, BITNEST_PATH_AUTO, stream);
+}
+
+int bitnest_debug_group_sums(int mode, const uint8_t *hi, const uint8_t *lo,
+                             const int8_t *xq, const int32_t *xsum, int64_t M, int64_t N,
+                             int64_t K, int32_t *S, int path, void *stream) {
+  if (path < BITNEST_PATH_AUTO || path > BITNEST_PATH_TC) return BITNEST_ERR_INVALID_ARG;
+  if (mode != BITNEST_DRAFT && mode != BITNEST_TARGET) return BITNEST_ERR_INVALID_ARG;
+  int s = check_shape(M, N, K);
+  if (s != BITNEST_OK) return s;
+  if (M == 0 || N == 0) return BITNEST_OK;
+  if (!hi || !xq || !xsum || !S || (mode == BITNEST_TARGET && !lo))
+    return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(hi) || misaligned(xq) || misaligned(xsum) || misaligned(S) ||
+      (mode == BITNEST_TARGET && misaligned(lo)))
+    return BITNEST_ERR_MISALIGNED;
+  if (M == 0 || N == 0) return BITNEST_OK;
+  LinearArgs a{mode, hi, mode == BITNEST_TARGET ? lo : nullptr, nullptr, xq, nullptr, xsum,
+               nullptr, nullptr, S, M, N, K, 0};
+  return run_linear(a, path, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,42 @@
+// Internal launchers (C++), called only by the C ABI in capi.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bitnest {
+
+struct LinearArgs {
+  int mode;               // 0 draft, 1 target
+  const uint8_t *hi;      // [N, K/2]
+  const uint8_t *lo;      // [N, K/2] (target)
+  const uint16_t *scale;  // fp16 [N, K/128]
+  const int8_t *xq;       // [M, K]
+  const float *xscale;    // [M] or [M, K/128]
+  const int32_t *xsum;    // [M, K/128]
+  const uint16_t *bias;   // fp16 [N] or null
+  float *y;               // [M, N]
+  int32_t *S;             // debug group sums [M, N, K/128] (null unless debug)
+  int64_t M, N, K;
+  int act_group;          // 0 or 128
+};
+
+cudaError_t launch_pack(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K, uint8_t *hi,
+                        uint8_t *lo, cudaStream_t st);
+cudaError_t launch_quantize(const uint16_t *x, int64_t M, int64_t K, int act_group, int8_t *xq,
+                            float *xs, int32_t *xsum, cudaStream_t st);
+cudaError_t launch_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
+                                  cudaStream_t st);
+
+// Largest M * K the GEMV kernels can stage in shared memory.
+bool gemv_fits(int64_t M, int64_t K);
+cudaError_t launch_gemv(const LinearArgs &a, cudaStream_t st);
+
+// tcgen05 tensor-core GEMM (any M).
+bool tc_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_tc(const LinearArgs &a, cudaStream_t st);
+
+// The flag a bounded wait sets when it gives up (synchronous read).
+cudaError_t read_wait_timeout(int *flag, bool reset);
+
+}  // namespace bitnest

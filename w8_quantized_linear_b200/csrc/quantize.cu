@@ -1,0 +1,169 @@
+// Plane packing, symmetric int8 activation quantisation and activation group
+// sums.  BitNest-Llama-3-8B model card: section "Files" (plane layout) and the
+// model table row "Activations" (symmetric int8 per token, per 128-group for
+// o_proj).
+#include "common.cuh"
+#include "launch.h"
+
+namespace bitnest {
+
+// ---------------------------------------------------------------- packing
+// Each thread writes 4 plane bytes from 8 nibbles of one row.
+__global__ void pack_kernel(const uint8_t *__restrict__ u, int64_t total_words,
+                            uint8_t *__restrict__ plane) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= total_words) return;
+  const uint2 v = *reinterpret_cast<const uint2 *>(u + 8 * i);  // columns 8i .. 8i+7
+  // t: byte b = u[b] & 15; t | t >> 4 puts u[2j] | u[2j+1] << 4 in byte 2j
+  uint32_t a = v.x & 0x0F0F0F0Fu, b = v.y & 0x0F0F0F0Fu;
+  a |= a >> 4;
+  b |= b >> 4;
+  reinterpret_cast<uint32_t *>(plane)[i] = prmt(a, b, 0x6420);
+}
+
+cudaError_t launch_pack(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K, uint8_t *hi,
+                        uint8_t *lo, cudaStream_t st) {
+  int64_t words = N * K / 8;
+  int threads = 256;
+  int64_t blocks = (words + threads - 1) / threads;
+  pack_kernel<<<(unsigned)blocks, threads, 0, st>>>(uh, words, hi);
+  if (ul && lo) pack_kernel<<<(unsigned)blocks, threads, 0, st>>>(ul, words, lo);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ quantiser
+// q = clamp(rne(x / s), -127, 127), s = max|x| / 127 (correctly rounded fp32
+// division); s == 0 gives q = 0.
+__device__ __forceinline__ int quant_one(float x, float s) {
+  if (s == 0.0f) return 0;
+  int q = __float2int_rn(__fdiv_rn(x, s));
+  return max(-127, min(127, q));
+}
+
+// Quantise 8 values (one 16-byte vector); returns the 8 codes packed and
+// adds their sum to *sum.
+__device__ __forceinline__ uint2 quant8(const uint4 v, float s, int *sum) {
+  const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __half22float2(h[i]);
+    int q0 = quant_one(f.x, s), q1 = quant_one(f.y, s);
+    *sum += q0 + q1;
+    uint32_t pair = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8);
+    w[i >> 1] |= pair << (16 * (i & 1));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ float amax8(const uint4 v) {
+  const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __half22float2(h[i]);
+    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+  }
+  return m;
+}
+
+// One block per token.  Vector v (8 columns) is handled by thread v % T; a
+// group (16 vectors) is 16 consecutive threads of one pass.
+template <int T>
+__global__ void __launch_bounds__(T) quantize_token_kernel(const uint16_t *__restrict__ x,
+                                                           int64_t K, int8_t *__restrict__ xq,
+                                                           float *__restrict__ xs,
+                                                           int32_t *__restrict__ xsum) {
+  const int64_t m = blockIdx.x;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + m * K);
+  const int nvec = (int)(K / 8);
+  float amax = 0.0f;
+  for (int v = threadIdx.x; v < nvec; v += T) amax = fmaxf(amax, amax8(__ldg(xr + v)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  __shared__ float red[T / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < T / 32; ++i) amax = fmaxf(amax, red[i]);
+  const float s = __fdiv_rn(amax, 127.0f);
+  if (threadIdx.x == 0) xs[m] = s;
+  uint2 *qr = reinterpret_cast<uint2 *>(xq + m * K);
+  const int G = (int)(K / kGroup);
+  for (int v0 = 0; v0 < nvec; v0 += T) {
+    const int v = v0 + threadIdx.x;
+    int sum = 0;
+    if (v < nvec) qr[v] = quant8(__ldg(xr + v), s, &sum);
+    // 16 consecutive threads hold one group (T is a multiple of 16, nvec of 16)
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (xsum && v < nvec && (v & 15) == 0) xsum[m * G + v / 16] = sum;
+  }
+}
+
+// act_group = 128: 16 threads per group, one scale per (token, group).
+__global__ void __launch_bounds__(256) quantize_group_kernel(const uint16_t *__restrict__ x,
+                                                             int64_t M, int64_t K,
+                                                             int8_t *__restrict__ xq,
+                                                             float *__restrict__ xs,
+                                                             int32_t *__restrict__ xsum) {
+  const int64_t nvec = M * K / 8;
+  const int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // vectors in order
+  const bool ok = v < nvec;  // nvec is a multiple of 16: whole groups share `ok`
+  uint4 val = ok ? __ldg(reinterpret_cast<const uint4 *>(x) + v) : make_uint4(0, 0, 0, 0);
+  float amax = amax8(val);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = __fdiv_rn(amax, 127.0f);
+  int sum = 0;
+  uint2 q = quant8(val, s, &sum);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (ok) {
+    reinterpret_cast<uint2 *>(xq)[v] = q;
+    if ((v & 15) == 0) {
+      const int64_t grp = v / 16;  // = m * G + g
+      xs[grp] = s;
+      if (xsum) xsum[grp] = sum;
+    }
+  }
+}
+
+cudaError_t launch_quantize(const uint16_t *x, int64_t M, int64_t K, int act_group, int8_t *xq,
+                            float *xs, int32_t *xsum, cudaStream_t st) {
+  if (act_group == 0) {
+    quantize_token_kernel<512><<<(unsigned)M, 512, 0, st>>>(x, K, xq, xs, xsum);
+  } else {
+    const int64_t nvec = M * K / 8;
+    const int threads = 256;
+    quantize_group_kernel<<<(unsigned)((nvec + threads - 1) / threads), threads, 0, st>>>(
+        x, M, K, xq, xs, xsum);
+  }
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------ activation sums
+// One warp per (token, group): 128 bytes, 4 per lane.
+__global__ void act_group_sums_kernel(const int8_t *__restrict__ xq, int64_t groups,
+                                      int32_t *__restrict__ xsum) {
+  const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= groups) return;
+  const uint32_t word = reinterpret_cast<const uint32_t *>(xq + w * kGroup)[lane];
+  int sum = __dp4a((int)word, 0x01010101, 0);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) xsum[w] = sum;
+}
+
+cudaError_t launch_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
+                                  cudaStream_t st) {
+  const int64_t groups = M * (K / kGroup);
+  const int threads = 256;
+  const int64_t blocks = (groups * 32 + threads - 1) / threads;
+  act_group_sums_kernel<<<(unsigned)blocks, threads, 0, st>>>(xq, groups, xsum);
+  return cudaGetLastError();
+}
+
+}  // namespace bitnest
