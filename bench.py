@@ -253,6 +253,49 @@ def timed_replays(graphs, steps, barrier):
     return start.elapsed_time(end) / 1e3  # seconds
 
 
+# ----------------------------------------------------------------- prefill
+PREFILL_M = 2048
+
+
+def measure_prefill(wl, reps=10):
+    """Target W8A8 at M = 2048 through the seven projections on the tcgen05
+    path.  Each launch is timed alone with CUDA events after an L2 flush
+    (a 256 MB write); returns per-projection and total int8 TOPS."""
+    import torch
+
+    bn = wl.bn
+    dev = wl.dev
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    tot_ops = 0.0
+    tot_t = 0.0
+    for name, (N, K, g) in wl.projs:
+        pid = synth.PROJ_IDS[name]
+        x = torch.from_numpy(synth.activations(synth.SEED_ACTS + pid, PREFILL_M, K)).to(dev)
+        xq, xs, xsum = bn.quantize_act(x, g)
+        y = torch.empty((PREFILL_M, N), dtype=torch.float32, device=dev)
+        hi, lo, sc = wl.copies[0][name]
+        bn.linear(1, hi, lo, sc, xq, xs, xsum, g, out=y)  # warm
+        t = 0.0
+        for _ in range(reps):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            bn.linear(1, hi, lo, sc, xq, xs, xsum, g, out=y)
+            b.record()
+            torch.cuda.synchronize()
+            t += a.elapsed_time(b) / 1e3
+        t /= reps
+        ops = 2.0 * PREFILL_M * N * K
+        res[name] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1)}
+        tot_ops += ops
+        tot_t += t
+        del x, xq, xs, xsum, y
+    del flush
+    return res, tot_ops, tot_t
+
+
 # -------------------------------------------------------------- CPU oracle
 def cpu_baseline(rows_per_proj=256, budget_s=20.0):
     """The oracle, as it stands, on the host cores: every projection and both
@@ -280,6 +323,82 @@ def cpu_baseline(rows_per_proj=256, budget_s=20.0):
     return t_total, oracle.num_threads(), sampled
 
 
+def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind):
+    """The timed decode step (CUDA graphs over rotating weight copies), the
+    end-to-end variant with host buffers, and per-launch kernel times."""
+    import torch
+
+    step_bytes = wl.step_bytes()
+    graphs = [capture(lambda c=c: wl.run_step(c)) for c in range(N_COPIES)]
+    e2e_graphs = [capture(lambda c=c: wl.run_step(c, e2e=True)) for c in range(N_COPIES)]
+
+    for i in range(args.warmup):
+        graphs[i % N_COPIES].replay()
+    torch.cuda.synchronize()
+
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t = timed_replays(graphs, args.steps, barrier)
+    t = max_over_ranks(t)
+    ms_per_step = 1e3 * t / args.steps
+    value = world * step_bytes * args.steps / t / 1e9
+
+    # end to end: activations uploaded from pinned host memory and outputs read back
+    for i in range(args.warmup):
+        e2e_graphs[i % N_COPIES].replay()
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(timed_replays(e2e_graphs, args.steps, barrier))
+    e2e_value = world * step_bytes * args.steps / t_e2e / 1e9
+    h2d, d2h = wl.io_bytes()
+
+    # dominant kernel: the verify (target, M = 4) GEMV.  Per-launch device
+    # time from CUDA events recorded on the launching stream right around each
+    # launch; a spin kernel first lets the host enqueue the whole sequence, so
+    # no launch waits on the host between its two events.
+    events = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for k in wl.bufs}
+    dur = {k: 0.0 for k in events}
+    n_ev = max(8, min(args.steps, 200))
+    for i in range(n_ev):
+        torch.cuda._sleep(4_000_000)
+        wl.run_step(i % N_COPIES, events=events)
+        torch.cuda.synchronize()
+        for k, (a, b) in events.items():
+            dur[k] += a.elapsed_time(b) / 1e3
+    target_keys = [k for k in events if k[1] == 1]
+    draft_keys = [k for k in events if k[1] == 0]
+    tgt_bytes = sum(linear_bytes(1, 4, *synth.LLAMA3_8B_PROJECTIONS[k[0]][:2]) for k in target_keys)
+    tgt_time = sum(dur[k] for k in target_keys) / n_ev
+    drf_bytes = sum(linear_bytes(0, 1, *synth.LLAMA3_8B_PROJECTIONS[k[0]][:2]) for k in draft_keys)
+    drf_time = sum(dur[k] for k in draft_keys) / n_ev
+    per_proj = {}
+    for (name, mode) in events:
+        N, K, _ = synth.LLAMA3_8B_PROJECTIONS[name]
+        d = dur[name, mode] / n_ev
+        b = linear_bytes(mode, DECODE_M[mode], N, K)
+        per_proj[f"{name}/{'draft' if mode == 0 else 'target'}"] = {
+            "us": round(d * 1e6, 3), "GB/s": round(b / d / 1e9, 1),
+            "frac_hbm": round(b / d / 1e9 / hbm_peak, 3)}
+    achieved = tgt_bytes / tgt_time / 1e9
+    roofline = {
+        "bound": "hbm",
+        "kernel": "gemv_kernel<TARGET, M=4> (7 projections)",
+        "achieved": round(achieved, 1),
+        "peak": hbm_peak,
+        "unit": "GB/s",
+        "frac": round(achieved / hbm_peak, 4),
+        "peak_kind": f"{peak_kind} (copy bandwidth)",
+        "traffic": dominant_traffic("gemv_target_m4"),
+        "algorithmic_bytes_per_launch": round(tgt_bytes / len(target_keys)),
+        "draft_gemv_achieved": round(drf_bytes / drf_time / 1e9, 1),
+        "draft_gemv_frac": round(drf_bytes / drf_time / 1e9 / hbm_peak, 4),
+        "per_projection": per_proj,
+    }
+    for g in graphs + e2e_graphs:
+        g.reset()
+    return value, ms_per_step, clocks, e2e_value, h2d, d2h, roofline
+
+
+
 # ------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -288,6 +407,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="bitnest", choices=["bitnest", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="all", choices=["all", "decode", "prefill"],
+                    help="all: the decode step line with the prefill object; decode / "
+                         "prefill: only that part (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -324,73 +446,34 @@ def main():
 
     wl = DecodeWorkload(device)
     step_bytes = wl.step_bytes()
-    graphs = [capture(lambda c=c: wl.run_step(c)) for c in range(N_COPIES)]
-    e2e_graphs = [capture(lambda c=c: wl.run_step(c, e2e=True)) for c in range(N_COPIES)]
-
-    for i in range(args.warmup):
-        graphs[i % N_COPIES].replay()
-    torch.cuda.synchronize()
-
-    with ClockSampler(local_rank) as clocks:
-        t = timed_replays(graphs, args.steps, barrier)
-    t = max_over_ranks(t)
-    ms_per_step = 1e3 * t / args.steps
-    value = world * step_bytes * args.steps / t / 1e9
-
-    # end to end: activations uploaded from pinned host memory and outputs read back
-    for i in range(args.warmup):
-        e2e_graphs[i % N_COPIES].replay()
-    torch.cuda.synchronize()
-    t_e2e = max_over_ranks(timed_replays(e2e_graphs, args.steps, barrier))
-    e2e_value = world * step_bytes * args.steps / t_e2e / 1e9
-    h2d, d2h = wl.io_bytes()
-
-    # dominant kernel: the verify (target, M = 4) GEMV.  Per-launch device
-    # time from CUDA events recorded on the launching stream right around each
-    # launch; a spin kernel first lets the host enqueue the whole sequence, so
-    # no launch waits on the host between its two events.
-    events = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for k in wl.bufs}
-    dur = {k: 0.0 for k in events}
-    n_ev = max(8, min(args.steps, 200))
-    for i in range(n_ev):
-        torch.cuda._sleep(400_000)
-        wl.run_step(i % N_COPIES, events=events)
-        torch.cuda.synchronize()
-        for k, (a, b) in events.items():
-            dur[k] += a.elapsed_time(b) / 1e3
-    target_keys = [k for k in events if k[1] == 1]
-    draft_keys = [k for k in events if k[1] == 0]
-    tgt_bytes = sum(linear_bytes(1, 4, *synth.LLAMA3_8B_PROJECTIONS[k[0]][:2]) for k in target_keys)
-    tgt_time = sum(dur[k] for k in target_keys) / n_ev
-    drf_bytes = sum(linear_bytes(0, 1, *synth.LLAMA3_8B_PROJECTIONS[k[0]][:2]) for k in draft_keys)
-    drf_time = sum(dur[k] for k in draft_keys) / n_ev
     hbm_peak, bf16_peak, peak_kind = load_peaks()
-    per_proj = {}
-    for (name, mode) in events:
-        N, K, _ = synth.LLAMA3_8B_PROJECTIONS[name]
-        d = dur[name, mode] / n_ev
-        b = linear_bytes(mode, DECODE_M[mode], N, K)
-        per_proj[f"{name}/{'draft' if mode == 0 else 'target'}"] = {
-            "us": round(d * 1e6, 3), "GB/s": round(b / d / 1e9, 1),
-            "frac_hbm": round(b / d / 1e9 / hbm_peak, 3)}
-    achieved = tgt_bytes / tgt_time / 1e9
-    roofline = {
-        "bound": "hbm",
-        "kernel": "gemv_kernel<TARGET, M=4> (7 projections)",
-        "achieved": round(achieved, 1),
-        "peak": hbm_peak,
-        "unit": "GB/s",
-        "frac": round(achieved / hbm_peak, 4),
-        "peak_kind": f"{peak_kind} (copy bandwidth)",
-        "traffic": dominant_traffic("gemv_target_m4"),
-        "algorithmic_bytes_per_launch": round(tgt_bytes / len(target_keys)),
-        "draft_gemv_achieved": round(drf_bytes / drf_time / 1e9, 1),
-        "draft_gemv_frac": round(drf_bytes / drf_time / 1e9 / hbm_peak, 4),
-        "per_projection": per_proj,
-    }
-    for g in graphs + e2e_graphs:
-        g.reset()
+    dec = None
+    if args.workload in ("all", "decode"):
+        dec = measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind)
+    prefill = None
+    if args.workload in ("all", "prefill"):
+        pre, pre_ops, pre_t = measure_prefill(wl, reps=10 if args.workload == "all" else 3)
+        int8_peak = 2.0 * bf16_peak  # dense int8 : dense bf16 = 2 : 1 (nominal 4.5 : 2.25 PFLOP/s)
+        pre_tops = pre_ops / pre_t / 1e12
+        prefill = {
+            "workload": f"target W8A8, M={PREFILL_M}, 7 Llama-3-8B-shaped projections, tcgen05 kind::i8",
+            "TOPS": round(pre_tops, 1),
+            "us_total": round(pre_t * 1e6, 1),
+            "roofline": {"bound": "tensor", "achieved": round(pre_tops, 1),
+                         "peak": round(int8_peak, 1), "unit": "TOPS",
+                         "frac": round(pre_tops / int8_peak, 4),
+                         "peak_kind": f"{peak_kind} bf16 x 2 (dense int8 : bf16 nominal ratio)"},
+            "per_projection": pre,
+            "l2": "flushed (256 MB write) before every timed launch",
+        }
+    if dec is None:
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "workload": "prefill only", "prefill": prefill}),
+                  flush=True)
+        return
+    value, ms_per_step, clocks, e2e_value, h2d, d2h, roofline = dec
 
     out = {
         "metric": METRIC,
@@ -423,6 +506,8 @@ def main():
         "gpu_launches": wl.launches_per_step() * args.steps,
         "roofline": roofline,
     }
+    if prefill is not None:
+        out["prefill"] = prefill
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, cores, rows = cpu_baseline()
         out["cpu_baseline"] = {
