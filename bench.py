@@ -142,88 +142,164 @@ def dominant_traffic(kernel_tag):
 
 
 # ---------------------------------------------------------------- workload
-class DecodeWorkload:
-    """Weights (N_COPIES rotating copies), activations and outputs on one GPU."""
+# One decoder layer's projections as launched by an inference engine: q|k|v
+# share their input and are one fused weight (N = 6144), likewise gate|up
+# (N = 28672); o_proj takes per-128-group activation scales.
+LAYER_GROUPS = [
+    ("qkv", ("q_proj", "k_proj", "v_proj")),
+    ("o", ("o_proj",)),
+    ("gate_up", ("gate_proj", "up_proj")),
+    ("down", ("down_proj",)),
+]
 
-    def __init__(self, device, n_copies=N_COPIES):
+
+def group_shape(members):
+    N = sum(synth.LLAMA3_8B_PROJECTIONS[m][0] for m in members)
+    K = synth.LLAMA3_8B_PROJECTIONS[members[0]][1]
+    g = synth.LLAMA3_8B_PROJECTIONS[members[0]][2]
+    return N, K, g
+
+
+def decode_step_bytes():
+    """Algorithmic bytes of one decode step (both passes, all layer groups)."""
+    tot = 0
+    for _, members in LAYER_GROUPS:
+        N, K, g = group_shape(members)
+        for mode, M in DECODE_M.items():
+            tot += linear_bytes(mode, M, N, K) + quant_bytes(M, K, g)
+    return tot
+
+
+class DecodeWorkload:
+    """Weights (N_COPIES rotating copies of the fused layer weights, plus one
+    unfused copy for per-projection timing), activations and outputs."""
+
+    def __init__(self, device, n_copies=N_COPIES, overlap=True):
         import torch
 
         import w8_quantized_linear_b200 as bn
 
         self.bn = bn
+        self.overlap = overlap
         self.dev = device
         self.projs = list(synth.LLAMA3_8B_PROJECTIONS.items())
-        self.copies = []  # per copy: {name: (hi, lo, scale)}
-        base = {}
+        nib = {}
         for name, (N, K, _) in self.projs:
             pid = synth.PROJ_IDS[name]
-            uh = torch.from_numpy(synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K))
-            ul = torch.from_numpy(synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K))
-            hi, lo = bn.pack_planes(uh.to(device), ul.to(device))
-            s = torch.from_numpy(synth.group_scales(synth.SEED_SCALES + pid, N, K)).to(device)
-            base[name] = (hi, lo, s)
-        self.copies.append(base)
-        for _ in range(1, n_copies):
-            self.copies.append({k: tuple(t.clone() for t in v) for k, v in base.items()})
-        # activations (fp16, device and pinned host) and the buffers of the step
-        self.x = {}
-        self.x_host = {}
-        self.bufs = {}
+            nib[name] = (synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K),
+                         synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K),
+                         synth.group_scales(synth.SEED_SCALES + pid, N, K))
+
+        def planes(uh, ul, s):
+            hi, lo = bn.pack_planes(torch.from_numpy(uh).to(device), torch.from_numpy(ul).to(device))
+            return hi, lo, torch.from_numpy(s).to(device)
+
+        self.single = {name: planes(*nib[name]) for name, _ in self.projs}
+        base = {}
+        for gname, members in LAYER_GROUPS:
+            base[gname] = planes(*(np.concatenate([nib[m][i] for m in members], axis=0)
+                                   for i in range(3)))
+        self.copies = [base] + [{k: tuple(t.clone() for t in v) for k, v in base.items()}
+                                for _ in range(1, n_copies)]
+        # per layer group and pass: activations (device and pinned host) and buffers
+        self.x, self.x_host, self.bufs = {}, {}, {}
+        for gi, (gname, members) in enumerate(LAYER_GROUPS):
+            N, K, g = group_shape(members)
+            for mode, M in DECODE_M.items():
+                xh = torch.from_numpy(synth.activations(synth.SEED_ACTS + 10 * gi + 100 * mode, M, K))
+                self.x_host[gname, mode] = xh.pin_memory()
+                self.x[gname, mode] = xh.to(device)
+                self.bufs[gname, mode] = self._bufs(M, N, K, g)
+        # unfused per-projection buffers (kernel timing)
+        self.pbufs = {}
         for name, (N, K, g) in self.projs:
             pid = synth.PROJ_IDS[name]
             for mode, M in DECODE_M.items():
-                xh = torch.from_numpy(synth.activations(synth.SEED_ACTS + pid + 100 * mode, M, K))
-                self.x_host[name, mode] = xh.pin_memory()
-                self.x[name, mode] = xh.to(device)
-                G = K // 128
-                self.bufs[name, mode] = dict(
-                    xq=torch.empty((M, K), dtype=torch.int8, device=device),
-                    xs=torch.empty((M,) if g == 0 else (M, G), dtype=torch.float32, device=device),
-                    xsum=torch.empty((M, G), dtype=torch.int32, device=device),
-                    y=torch.empty((M, N), dtype=torch.float32, device=device),
-                    y_host=torch.empty((M, N), dtype=torch.float32).pin_memory(),
-                )
+                x = torch.from_numpy(synth.activations(synth.SEED_ACTS + pid + 100 * mode, M, K))
+                self.pbufs[name, mode] = dict(self._bufs(M, N, K, g), x=x.to(device))
         torch.cuda.synchronize()
 
+    def _bufs(self, M, N, K, g):
+        import torch
+
+        G = K // 128
+        return dict(
+            xq=torch.empty((M, K), dtype=torch.int8, device=self.dev),
+            xs=torch.empty((M,) if g == 0 else (M, G), dtype=torch.float32, device=self.dev),
+            xsum=torch.empty((M, G), dtype=torch.int32, device=self.dev),
+            y=torch.empty((M, N), dtype=torch.float32, device=self.dev),
+            y_host=torch.empty((M, N), dtype=torch.float32).pin_memory(),
+        )
+
     def step_bytes(self):
-        tot = 0
-        for name, (N, K, g) in self.projs:
-            for mode, M in DECODE_M.items():
-                tot += linear_bytes(mode, M, N, K) + quant_bytes(M, K, g)
-        return tot
+        return decode_step_bytes()
 
     def launches_per_step(self):
-        return 2 * 2 * len(self.projs)
+        return 2 * 2 * len(LAYER_GROUPS)
 
     def io_bytes(self):
         h2d = sum(t.numel() * t.element_size() for t in self.x_host.values())
         d2h = sum(b["y_host"].numel() * 4 for b in self.bufs.values())
         return h2d, d2h
 
+    def _path(self):
+        return self.bn.PATH_AUTO | (self.bn.PATH_OVERLAP if self.overlap else 0)
+
     def run_step(self, copy, events=None, e2e=False):
-        """Enqueue one step on the current stream; `events`: per (name, mode)
-        (start, end) CUDA events recorded around each linear launch."""
+        """Enqueue one step on the current stream: the draft pass then the
+        verify pass, each quantise + linear for the four layer groups.
+        `events`: per (group, mode) (start, end) CUDA events around the linear."""
         bn = self.bn
         w = self.copies[copy]
         for mode in (0, 1):
-            for name, (N, K, g) in self.projs:
-                b = self.bufs[name, mode]
-                x = self.x[name, mode]
+            for gname, members in LAYER_GROUPS:
+                _, _, g = group_shape(members)
+                b = self.bufs[gname, mode]
+                x = self.x[gname, mode]
                 if e2e:
-                    x.copy_(self.x_host[name, mode], non_blocking=True)
+                    x.copy_(self.x_host[gname, mode], non_blocking=True)
                 bn.quantize_act(x, g, out=(b["xq"], b["xs"], b["xsum"]))
-                hi, lo, s = w[name]
+                hi, lo, s = w[gname]
                 if events is not None:
-                    events[name, mode][0].record()
-                bn.linear(mode, hi, lo, s, b["xq"], b["xs"], b["xsum"], g, out=b["y"])
+                    events[gname, mode][0].record()
+                bn.linear(mode, hi, lo, s, b["xq"], b["xs"], b["xsum"], g, out=b["y"],
+                          path=self._path())
                 if events is not None:
-                    events[name, mode][1].record()
+                    events[gname, mode][1].record()
                 if e2e:
                     b["y_host"].copy_(b["y"], non_blocking=True)
 
+    def run_projection(self, name, mode):
+        """One unfused projection: quantise its own input, then the linear."""
+        bn = self.bn
+        _, _, g = synth.LLAMA3_8B_PROJECTIONS[name]
+        b = self.pbufs[name, mode]
+        bn.quantize_act(b["x"], g, out=(b["xq"], b["xs"], b["xsum"]))
+        hi, lo, s = self.single[name]
+        return lambda: bn.linear(mode, hi, lo, s, b["xq"], b["xs"], b["xsum"], g, out=b["y"],
+                                 path=self._path())
 
-def capture(fn):
+
+class EagerStep:
+    """Stands in for a captured graph: replay() launches the step directly."""
+
+    def __init__(self, fn):
+        self.fn = fn
+
+    def replay(self):
+        self.fn()
+
+    def reset(self):
+        pass
+
+
+def capture(fn, eager=False):
     import torch
+
+    if eager:
+        fn()
+        torch.cuda.synchronize()
+        return EagerStep(fn)
 
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
@@ -329,8 +405,9 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
     import torch
 
     step_bytes = wl.step_bytes()
-    graphs = [capture(lambda c=c: wl.run_step(c)) for c in range(N_COPIES)]
-    e2e_graphs = [capture(lambda c=c: wl.run_step(c, e2e=True)) for c in range(N_COPIES)]
+    eager = args.no_graph
+    graphs = [capture(lambda c=c: wl.run_step(c), eager) for c in range(N_COPIES)]
+    e2e_graphs = [capture(lambda c=c: wl.run_step(c, e2e=True), eager) for c in range(N_COPIES)]
 
     for i in range(args.warmup):
         graphs[i % N_COPIES].replay()
@@ -364,34 +441,51 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
         torch.cuda.synchronize()
         for k, (a, b) in events.items():
             dur[k] += a.elapsed_time(b) / 1e3
-    target_keys = [k for k in events if k[1] == 1]
-    draft_keys = [k for k in events if k[1] == 0]
-    tgt_bytes = sum(linear_bytes(1, 4, *synth.LLAMA3_8B_PROJECTIONS[k[0]][:2]) for k in target_keys)
-    tgt_time = sum(dur[k] for k in target_keys) / n_ev
-    drf_bytes = sum(linear_bytes(0, 1, *synth.LLAMA3_8B_PROJECTIONS[k[0]][:2]) for k in draft_keys)
-    drf_time = sum(dur[k] for k in draft_keys) / n_ev
-    per_proj = {}
-    for (name, mode) in events:
-        N, K, _ = synth.LLAMA3_8B_PROJECTIONS[name]
-        d = dur[name, mode] / n_ev
+    per_group = {}
+    for (gname, mode) in events:
+        N, K, _ = group_shape(dict(LAYER_GROUPS)[gname])
+        d = dur[gname, mode] / n_ev
         b = linear_bytes(mode, DECODE_M[mode], N, K)
-        per_proj[f"{name}/{'draft' if mode == 0 else 'target'}"] = {
-            "us": round(d * 1e6, 3), "GB/s": round(b / d / 1e9, 1),
+        per_group[f"{gname}/{'draft' if mode == 0 else 'target'}"] = {
+            "N": N, "K": K, "us": round(d * 1e6, 3), "GB/s": round(b / d / 1e9, 1),
             "frac_hbm": round(b / d / 1e9 / hbm_peak, 3)}
-    achieved = tgt_bytes / tgt_time / 1e9
+    # the dominant launch: the fused gate|up verify (target, M = 4) linear
+    N, K, _ = group_shape(dict(LAYER_GROUPS)["gate_up"])
+    dom_bytes = linear_bytes(1, DECODE_M[1], N, K)
+    dom_time = dur["gate_up", 1] / n_ev
+    achieved = dom_bytes / dom_time / 1e9
+    # every projection on its own (unfused), same events
+    per_proj = {}
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for name, (N, K, _) in wl.projs:
+        for mode, M in DECODE_M.items():
+            t = 0.0
+            reps = 20
+            for _ in range(reps):
+                fn = wl.run_projection(name, mode)
+                torch.cuda._sleep(400_000)
+                ev0.record()
+                fn()
+                ev1.record()
+                torch.cuda.synchronize()
+                t += ev0.elapsed_time(ev1) / 1e3
+            t /= reps
+            b = linear_bytes(mode, M, N, K)
+            per_proj[f"{name}/{'draft' if mode == 0 else 'target'}"] = {
+                "us": round(t * 1e6, 3), "GB/s": round(b / t / 1e9, 1),
+                "frac_hbm": round(b / t / 1e9 / hbm_peak, 3)}
     roofline = {
         "bound": "hbm",
-        "kernel": "gemv_kernel<TARGET, M=4> (7 projections)",
+        "kernel": f"gemv_tma_kernel<TARGET, M=4>, fused gate|up (N={N}, K={K})",
         "achieved": round(achieved, 1),
         "peak": hbm_peak,
         "unit": "GB/s",
         "frac": round(achieved / hbm_peak, 4),
         "peak_kind": f"{peak_kind} (copy bandwidth)",
-        "traffic": dominant_traffic("gemv_target_m4"),
-        "algorithmic_bytes_per_launch": round(tgt_bytes / len(target_keys)),
-        "draft_gemv_achieved": round(drf_bytes / drf_time / 1e9, 1),
-        "draft_gemv_frac": round(drf_bytes / drf_time / 1e9 / hbm_peak, 4),
-        "per_projection": per_proj,
+        "traffic": dominant_traffic("gemv_target_m4_gate_up"),
+        "algorithmic_bytes_per_launch": dom_bytes,
+        "per_launch_in_step": per_group,
+        "per_projection_unfused": per_proj,
     }
     for g in graphs + e2e_graphs:
         g.reset()
@@ -407,6 +501,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="bitnest", choices=["bitnest", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch the layer kernels without programmatic dependent launch "
+                         "(ncu cannot replay such launches inside a captured graph)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the step's kernels directly instead of replaying a CUDA graph "
+                         "(for profilers that cannot replay the captured kernel nodes)")
     ap.add_argument("--workload", default="all", choices=["all", "decode", "prefill"],
                     help="all: the decode step line with the prefill object; decode / "
                          "prefill: only that part (for profiling runs)")
@@ -414,6 +514,8 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
+    if args.no_overlap:
+        os.environ["BITNEST_PDL"] = "0"  # read by the library at its first launch
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -444,7 +546,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    wl = DecodeWorkload(device)
+    wl = DecodeWorkload(device, overlap=not args.no_overlap)
     step_bytes = wl.step_bytes()
     hbm_peak, bf16_peak, peak_kind = load_peaks()
     dec = None
@@ -491,13 +593,16 @@ def main():
         "config": {
             "workload": wl_name,
             "projections": {k: list(v[:2]) for k, v in synth.LLAMA3_8B_PROJECTIONS.items()},
-            "passes": "draft W4A8 M=1 + target W8A8 M=4 per projection, quantise included",
+            "launches": "per pass: quantise + linear for q|k|v (fused, N=6144), o (per-group "
+                        "activation scales), gate|up (fused, N=28672), down",
+            "passes": "draft W4A8 M=1 then verify W8A8 M=4 (gamma+1)",
             "group": 128,
             "bytes_per_step": step_bytes,
-            "l2": f"inputs larger than L2: {N_COPIES} rotating weight copies "
+            "l2": f"inputs larger than L2: {N_COPIES} rotating copies of the layer weights "
                   f"({N_COPIES * sum(v[0] * v[1] for v in synth.LLAMA3_8B_PROJECTIONS.values()) / 1e6:.0f} MB of planes)",
             "parallelism": "replicas" if world > 1 else "single",
-            "timing": "CUDA graph per step, CUDA events on the launching stream",
+            "timing": ("direct launches" if args.no_graph else "CUDA graph per step")
+                      + ", CUDA events on the launching stream",
         },
         "clocks": clocks.summary(),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -526,10 +631,7 @@ def run_reference(args, rank, world, wl_name):
     """The oracle, as it stands, on the host cores (rank 0 only)."""
     if rank != 0:
         return
-    step_bytes = 0
-    for name, (N, K, g) in synth.LLAMA3_8B_PROJECTIONS.items():
-        for mode, M in DECODE_M.items():
-            step_bytes += linear_bytes(mode, M, N, K) + quant_bytes(M, K, g)
+    step_bytes = decode_step_bytes()
     rows = 64
     for _ in range(min(args.warmup, 1)):
         cpu_baseline(rows_per_proj=rows)

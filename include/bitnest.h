@@ -52,6 +52,18 @@ extern "C" {
 
 #define BITNEST_GEMV_MAX_M 8 /* largest M the GEMV kernels are built for */
 
+/* May be OR-ed into the `path` of bitnest_linear_path: the layer kernel is
+ * launched with programmatic dependent launch and starts streaming hi, lo and
+ * scale before the preceding kernel on the stream has finished; it waits for
+ * that kernel only before it reads xq / xscale / xsum.  Safe when no kernel
+ * still running on the stream writes the planes or the scales (a
+ * bitnest_quantize_act call right before is always safe: it waits for its own
+ * predecessor before it lets the next kernel start).  Setting the environment
+ * variable BITNEST_PDL=0 before the first call turns programmatic dependent
+ * launch off for every kernel of the library (profilers that replay captured
+ * graphs cannot replay such launches). */
+#define BITNEST_PATH_OVERLAP 0x100
+
 /* Status codes. */
 #define BITNEST_OK 0
 #define BITNEST_ERR_INVALID_ARG 1       /* null pointer, bad mode / group / path        */
@@ -131,8 +143,9 @@ int bitnest_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_
                    int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
                    void *stream);
 
-/* bitnest_linear with an explicit kernel family (BITNEST_PATH_*).  PATH_GEMV
- * requires M <= BITNEST_GEMV_MAX_M (else BITNEST_ERR_UNSUPPORTED_SHAPE). */
+/* bitnest_linear with an explicit kernel family (BITNEST_PATH_*, optionally
+ * OR-ed with BITNEST_PATH_OVERLAP).  PATH_GEMV requires M <= BITNEST_GEMV_MAX_M
+ * (else BITNEST_ERR_UNSUPPORTED_SHAPE). */
 int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
                         const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
                         int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,

@@ -183,3 +183,29 @@ def test_llama3_projection_decode_sampled(name):
         # the exact integer sums of the sampled rows
         S = host(bn.debug_group_sums(mode, d_hi, d_lo, d_xq, d_xsum))
         assert np.array_equal(S[:, rows, :], oracle.group_sums(mode, hi_rows, lo_rows, q, K))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (4, 1000, 2048), (3, 17, 14336), (8, 64, 1024)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gemv_overlap_launch(M, N, K, mode):
+    """Programmatic dependent launch after the quantiser gives the same result."""
+    p = Problem(M, N, K, seed=21 + M)
+    xq, xs, xsum = bn.quantize_act(p.d_x, 0)
+    y = bn.linear(mode, p.d_hi, p.d_lo, p.d_s, xq, xs, xsum,
+                  path=bn.PATH_GEMV | bn.PATH_OVERLAP)
+    torch.cuda.synchronize()
+    assert oracle.max_normalised_error(host(y), p.y_ref(mode)) <= TOL
+    assert bn.device_wait_timeout(reset=True) == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 3, 1024), (2, 9, 2048), (5, 200, 1024), (8, 130, 3072)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gemv_simple_kernel_for_odd_k(M, N, K, mode):
+    """K not a multiple of 1024 takes the plain-load GEMV; K that is takes the
+    TMA-ring GEMV: both agree with the oracle and with each other's sums."""
+    for KK in (K, K + 128):
+        p = Problem(M, N, KK, seed=KK + M)
+        S = bn.debug_group_sums(mode, p.d_hi, p.d_lo, p.d_xq, p.d_xsum, path=bn.PATH_GEMV)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(S), oracle.group_sums(mode, p.hi, p.lo, p.q, KK))
+        assert oracle.max_normalised_error(p.y_gpu(mode, bn.PATH_GEMV), p.y_ref(mode)) <= TOL

@@ -51,6 +51,7 @@ int pick_path(int mode, int64_t M, int64_t N, int64_t K) {
 int run_linear(const LinearArgs &a, int path, cudaStream_t st) {
   if (path == BITNEST_PATH_AUTO) path = pick_path(a.mode, a.M, a.N, a.K);
   if (path == BITNEST_PATH_GEMV) {
+    if (gemv_tma_supported(a.M, a.N, a.K)) return cuda_status(launch_gemv_tma(a, st));
     if (!gemv_fits(a.M, a.K)) return BITNEST_ERR_UNSUPPORTED_SHAPE;
     return cuda_status(launch_gemv(a, st));
   }
@@ -79,9 +80,10 @@ const char *bitnest_status_string(int status) {
 int bitnest_version(void) { return 100; }
 
 int bitnest_device_wait_timeout(int reset) {
-  int flag = 0;
-  if (read_wait_timeout(&flag, reset != 0) != cudaSuccess) return -BITNEST_ERR_CUDA;
-  return flag;
+  int f1 = 0, f2 = 0;
+  if (read_wait_timeout(&f1, reset != 0) != cudaSuccess) return -BITNEST_ERR_CUDA;
+  if (read_wait_timeout_gemv(&f2, reset != 0) != cudaSuccess) return -BITNEST_ERR_CUDA;
+  return (f1 | f2) ? 1 : 0;
 }
 
 int bitnest_pack_planes(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K,
@@ -128,12 +130,14 @@ int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const ui
                         const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
                         int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
                         int path, void *stream) {
+  const bool overlap = (path & BITNEST_PATH_OVERLAP) != 0;
+  path &= ~BITNEST_PATH_OVERLAP;
   if (path < BITNEST_PATH_AUTO || path > BITNEST_PATH_TC) return BITNEST_ERR_INVALID_ARG;
   int s = check_linear(mode, hi, lo, scale, xq, xscale, xsum, M, N, K, y, act_group, bias);
   if (s != BITNEST_OK) return s;
   if (M == 0 || N == 0) return BITNEST_OK;
   LinearArgs a{mode, hi, mode == BITNEST_TARGET ? lo : nullptr, scale, xq, xscale, xsum,
-               bias, y, nullptr, M, N, K, act_group};
+               bias, y, nullptr, M, N, K, act_group, overlap};
   return run_linear(a, path, (cudaStream_t)stream);
 }
 
@@ -160,7 +164,7 @@ int bitnest_debug_group_sums(int mode, const uint8_t *hi, const uint8_t *lo,
     return BITNEST_ERR_MISALIGNED;
   if (M == 0 || N == 0) return BITNEST_OK;
   LinearArgs a{mode, hi, mode == BITNEST_TARGET ? lo : nullptr, nullptr, xq, nullptr, xsum,
-               nullptr, nullptr, S, M, N, K, 0};
+               nullptr, nullptr, S, M, N, K, 0, false};
   return run_linear(a, path, (cudaStream_t)stream);
 }
 

@@ -4,6 +4,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 namespace bitnest {
 
@@ -44,6 +45,43 @@ template <>
 struct CodeOffset<1> {
   static constexpr int value = 136;
 };
+
+// Programmatic dependent launch: wait for the preceding kernel of the stream
+// (no-op when launched without the attribute) / let the next one start.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Programmatic dependent launch is used unless the environment variable
+// BITNEST_PDL is "0" (read once per process).
+inline bool pdl_enabled() {
+  static const int on = [] {
+    const char *v = getenv("BITNEST_PDL");
+    return (v && v[0] == '0' && v[1] == 0) ? 0 : 1;
+  }();
+  return on != 0;
+}
+
+// Launch `kern` with programmatic stream serialisation allowed when `pdl`.
+template <typename Kern, typename... Args>
+inline cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              bool pdl, Args... args) {
+  pdl = pdl && pdl_enabled();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

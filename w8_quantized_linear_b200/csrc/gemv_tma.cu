@@ -1,0 +1,568 @@
+// Decode GEMV of the bit-nested linear layer with a TMA shared-memory ring.
+//
+// BitNest-Llama-3-8B model card, section "Files": the draft reads the hi plane
+// only (W4 = (hi - 8) * scale); the target reads both planes
+// (W8 = (16 (hi - 8) + (lo - 8)) * scale / 16 = (((hi << 4) | lo) - 136) * scale / 16).
+//
+// The decode layer is a pure HBM stream: every weight byte is read once.  One
+// persistent CTA per SM.  A producer warp streams the CTA's 16-row blocks with
+// one TMA box per plane per stage (16 rows x 4096 columns = 32 KB, landed with
+// the 128-byte swizzle) into a ring of shared-memory stages.  On this part the
+// TMA streaming rate of an SM is set by a per-stage cost far more than by the
+// bytes, so stages are large and carry nothing else: the 16-bit group scales
+// are read by the consumers with 8-byte loads issued a stage ahead.
+//
+// Eight consumer warps each own four 128-column groups of a stage.  The
+// per-group integer sums go through the integer tensor-core MMA
+// (mma.sync m16n8k32, u8 weight bytes x s8 activations -> s32, 16 rows x 8
+// token slots x 32 columns): the weight byte is the nibble (draft) or
+// (hi << 4) | lo (target), unpacked in registers; the accumulator starts at
+// -offset * sum(q) of the group, so the MMA result is the exact group sum.
+// A dp4a inner loop needs about twice the issue slots of this and could not
+// keep up with HBM at 2 warps per scheduler.  The K-permutation that lets a
+// plane word's low / high nibbles feed the fragments without byte shuffles is
+// applied to the staged activations instead (even / odd columns).  Each warp
+// accumulates its groups' scaled sums in fp32; the 8 warps' partial sums of a
+// 16-row block are added in a fixed order by the last warp to finish it.
+//
+// With programmatic dependent launch the weight stream starts while the
+// preceding kernel (the activation quantiser) still runs; the consumers wait
+// for it (griddepcontrol.wait) before they read the activations.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace bitnest {
+namespace gv {
+
+constexpr int kConsumerWarps = 8;                      // four 128-column groups each per stage
+constexpr int kGroupsPerWarp = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;    // + one producer warp
+constexpr int kRows = 16;                              // weight rows per stage (the MMA's M)
+constexpr int kStepCols = 4096;                        // columns per stage = 32 groups
+constexpr int kSegs = kStepCols / 256;                 // 128-byte plane segments per row
+constexpr int kPlaneBytes = kRows * kStepCols / 2;     // 32 KB: one TMA box per plane
+constexpr int kMaxStages = 8;
+constexpr int kRedSlots = 2;  // row blocks whose partial sums can be in flight
+constexpr int kScaleSmemMax = 32 * 1024;  // the CTA's group scales are staged once
+constexpr int kSmemBudget = 227 * 1024;
+
+struct Params {
+  const uint16_t *scale;
+  const int8_t *xq;
+  const float *xscale;
+  const int32_t *xsum;
+  const uint16_t *bias;
+  float *y;
+  int32_t *S;
+  int M, N, K, G, Cp, Gp, nks, NB, stages;
+};
+
+__host__ __device__ constexpr int stage_bytes(int mode) { return (mode ? 2 : 1) * kPlaneBytes; }
+
+// row pitch (halves) of the staged group scales: an odd number of 8-byte
+// units, so rows stay 8-byte aligned and the 8 rows a warp reads with one
+// 8-byte load each fall in different banks
+__host__ __device__ inline int scale_pitch(int G) { return 4 * (((G + 3) / 4) | 1); }
+
+// staged activations [M][2][Cp] x 16 B, group sums [Gp][8], group act. scales
+// [Gp][8], the CTA's group scales [nb * 16][pitch] fp16, partial-sum slots
+// [kRedSlots][warps][128] and their counters
+__host__ __device__ inline int fixed_bytes(int M, int K, bool actg, int nb) {
+  const int nks = (K + kStepCols - 1) / kStepCols;
+  const int Cp = nks * (kStepCols / 32), Gp = nks * (kStepCols / kGroup);
+  const int G = K / kGroup;
+  int o = M * Cp * 32 + Gp * 32 + (actg ? Gp * 32 : 0) + (nb * kRows * scale_pitch(G) * 2 + 15) / 16 * 16 +
+          kRedSlots * kConsumerWarps * 128 * 4 + kRedSlots * 4;
+  return (o + 1023) / 1024 * 1024;
+}
+
+__host__ inline int smem_total(int mode, int M, bool actg, int K, int nb, int stages) {
+  return 1024 + fixed_bytes(M, K, actg, nb) + stages * stage_bytes(mode) +
+         (2 * kMaxStages + kRedSlots) * 8;
+}
+
+// D = A (16x32 u8) * B (32x8 s8) + C, int32.  Not volatile: a pure function
+// of its operands, so the compiler may interleave independent MMA chains.
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1, const int (&c)[4]) {
+  asm(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%11,%12,%13};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]),
+        "r"(c[2]), "r"(c[3]));
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, uint64_t *bar, int x,
+                                            int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// MMA row g (0..7) reads stage row perm(g) (and perm(g) + 8): rows whose
+// swizzle phases differ by 4 share a shared-memory wavefront, so the 16-byte
+// loads of a warp hit 32 different banks.
+__device__ __forceinline__ int perm_row(int g) { return (g >> 1) + ((g & 1) << 2); }
+
+// Asynchronous 4-byte copy global -> shared.
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint32_t w, int hi) {
+  return __half2float(__ushort_as_half((uint16_t)(hi ? (w >> 16) : (w & 0xFFFFu))));
+}
+
+
+template <int MODE, int M, bool ACTG, bool DEBUG>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemv_tma_kernel(const __grid_constant__ CUtensorMap tm_hi,
+                    const __grid_constant__ CUtensorMap tm_lo, const Params p) {
+  constexpr int OFF = CodeOffset<MODE>::value;
+  constexpr int STAGE = stage_bytes(MODE);
+  constexpr int GS = kStepCols / kGroup;  // groups per stage (32)
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int Cp = p.Cp, Gp = p.Gp, G = p.G, S = p.stages;
+  uint4 *xs4 = reinterpret_cast<uint4 *>(smem);                    // [M][2][Cp]
+  int32_t *sr = reinterpret_cast<int32_t *>(smem + M * Cp * 32);   // [Gp][8] group sums
+  float *sxg = reinterpret_cast<float *>(sr + Gp * 8);             // [Gp][8] group act. scales
+  const int nb = (p.NB - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int sp = scale_pitch(G);
+  __half *ssc = reinterpret_cast<__half *>(sxg + (ACTG ? Gp * 8 : 0));  // [nb * 16][sp]
+  float *red = reinterpret_cast<float *>(
+      reinterpret_cast<uint8_t *>(ssc) + (nb * kRows * sp * 2 + 15) / 16 * 16);  // [slots][warps][128]
+  int *cnt = reinterpret_cast<int *>(red + kRedSlots * kConsumerWarps * 128);  // [slots]
+  uint8_t *ring = smem + fixed_bytes(M, p.K, ACTG, nb);            // 1024-aligned stages
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + S * STAGE);
+  uint64_t *empty = full + kMaxStages;
+  uint64_t *slot_free = empty + kMaxStages;  // [kRedSlots]: partial-sum slot read out
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    for (int i = 0; i < kRedSlots; ++i) {
+      mbar_init(&slot_free[i], 1);
+      cnt[i] = 0;
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  griddep_launch_dependents();
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_hi);
+      if (MODE) prefetch_tmap(&tm_lo);
+      int it = 0;
+      bool ok = true;
+      for (int k = 0; k < nb && ok; ++k) {
+        const int row0 = ((int)blockIdx.x + k * (int)gridDim.x) * kRows;
+        for (int ks = 0; ks < p.nks; ++ks, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], STAGE);
+          uint8_t *st = ring + s * STAGE;
+          tma_load_3d(st, &tm_hi, &full[s], 0, row0, ks * kSegs);
+          if (MODE) tma_load_3d(st + kPlaneBytes, &tm_lo, &full[s], 0, row0, ks * kSegs);
+        }
+      }
+      if (!ok)  // gave up: let the copies already issued land before leaving
+        for (int i = (it > S ? it - S : 0); i < it; ++i) mbar_wait(&full[i % S], (i / S) & 1);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  constexpr int NT = kConsumerWarps * 32;
+  // The group scales of every row this CTA owns (32-bit words), copied
+  // asynchronously: all of them are in flight at once.  Like the planes they
+  // do not come from the preceding kernel, so this starts before the wait.
+  if (!DEBUG) {
+    const int wpr = G / 2;  // G is even (a multiple of 8)
+    for (int i = threadIdx.x; i < nb * kRows * wpr; i += NT) {
+      const int rl = i / wpr, wd = i - rl * wpr;
+      const int n = ((int)blockIdx.x + (rl / kRows) * (int)gridDim.x) * kRows + rl % kRows;
+      uint32_t *dst = reinterpret_cast<uint32_t *>(ssc + rl * sp) + wd;
+      if (n < p.N)
+        cp_async4(dst, reinterpret_cast<const uint32_t *>(p.scale + (int64_t)n * G) + wd);
+      else
+        *dst = 0u;
+    }
+  }
+  griddep_wait();  // the activations are written by the preceding kernel
+  const int C = p.K / 32;
+  // activations: every load of this thread first, then the permuted stores
+  constexpr int XB = 8;  // items per batch
+  for (int base = threadIdx.x; base < M * Cp; base += XB * NT) {
+    uint4 va[XB], vb[XB];
+#pragma unroll
+    for (int u = 0; u < XB; ++u) {
+      const int item = base + u * NT;
+      va[u] = make_uint4(0, 0, 0, 0);
+      vb[u] = make_uint4(0, 0, 0, 0);
+      if (item < M * Cp) {
+        const int m = item / Cp, c = item - m * Cp;
+        if (c < C) {  // zero padding past K
+          const uint4 *src = reinterpret_cast<const uint4 *>(p.xq + (int64_t)m * p.K + 32 * c);
+          va[u] = __ldg(src);
+          vb[u] = __ldg(src + 1);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < XB; ++u) {
+      const int item = base + u * NT;
+      if (item < M * Cp) {
+        const int m = item / Cp, c = item - m * Cp;
+        const uint32_t w[8] = {va[u].x, va[u].y, va[u].z, va[u].w,
+                               vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+        uint32_t e[4], o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          e[i] = prmt(w[2 * i], w[2 * i + 1], 0x6420);  // columns 8i + 0,2,4,6
+          o[i] = prmt(w[2 * i], w[2 * i + 1], 0x7531);  // columns 8i + 1,3,5,7
+        }
+        xs4[(m * 2 + 0) * Cp + c] = make_uint4(e[0], o[0], e[1], o[1]);
+        xs4[(m * 2 + 1) * Cp + c] = make_uint4(e[2], o[2], e[3], o[3]);
+      }
+    }
+  }
+  // group sums (and per-group activation scales), [Gp][8]
+  for (int base = threadIdx.x; base < Gp * 8; base += 4 * NT) {
+    int rv[4];
+    float xv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * NT;
+      const int g = i >> 3, m = i & 7;
+      const bool in = i < Gp * 8 && m < M && g < G;
+      rv[u] = in ? __ldg(p.xsum + m * G + g) : 0;
+      xv[u] = (ACTG && in) ? __ldg(p.xscale + m * G + g) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * NT;
+      if (i < Gp * 8) {
+        sr[i] = rv[u];
+        if (ACTG) sxg[i] = xv[u];
+      }
+    }
+  }
+  float xt0 = 0.0f, xt1 = 0.0f;  // token scales of this thread's two output columns
+  if (!ACTG && !DEBUG) {
+    const int t0 = 2 * (lane & 3);
+    xt0 = t0 < M ? __ldg(p.xscale + t0) : 0.0f;
+    xt1 = t0 + 1 < M ? __ldg(p.xscale + t0 + 1) : 0.0f;
+  }
+  cp_async_wait_all();
+  asm volatile("bar.sync 1, %0;" ::"r"(NT) : "memory");
+
+  const int gid = lane >> 2, tig = lane & 3;  // MMA fragment coordinates
+  const int r0 = perm_row(gid), r1 = r0 + 8;  // stage rows of this thread's A rows
+  const int tok0 = 2 * tig, tok1 = 2 * tig + 1;
+  // byte offset of this thread's 16-byte chunk of group jl (0..31), row r
+  auto chunk_off = [&](int jl, int r) {
+    const int seg = jl >> 1, c = ((jl & 1) << 2) + tig;
+    return seg * (kRows * 128) + r * 128 + ((c ^ (r & 7)) << 4);
+  };
+
+  // after a wait gives up, no more waits are attempted; the warp runs out its
+  // loops without work (there is no CTA barrier it could be left at)
+  bool ok = true;
+  int it = 0;
+  for (int k = 0; k < nb; ++k) {
+    const int row0 = ((int)blockIdx.x + k * (int)gridDim.x) * kRows;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int ks = 0; ks < p.nks && ok; ++ks, ++it) {
+      uint2 sc_cur0 = make_uint2(0, 0), sc_cur1 = make_uint2(0, 0);
+      if (!DEBUG) {  // this warp's four group scales of rows r0, r1
+        const int gq = ks * GS + warp * kGroupsPerWarp;
+        if (gq < G) {
+          sc_cur0 = *reinterpret_cast<const uint2 *>(ssc + (k * kRows + r0) * sp + gq);
+          sc_cur1 = *reinterpret_cast<const uint2 *>(ssc + (k * kRows + r1) * sp + gq);
+        }
+      }
+      const int s = it % S;
+      ok = mbar_wait_warp(&full[s], (it / S) & 1);
+      if (!ok) break;
+      const uint8_t *st = ring + s * STAGE;
+#pragma unroll
+      for (int q = 0; q < kGroupsPerWarp; ++q) {
+        const int jl = warp * kGroupsPerWarp + q;  // group within the stage
+        const int g = ks * GS + jl;                 // global group index
+        const int off0 = chunk_off(jl, r0), off1 = chunk_off(jl, r1);
+        const uint4 h0 = *reinterpret_cast<const uint4 *>(st + off0);
+        const uint4 h1 = *reinterpret_cast<const uint4 *>(st + off1);
+        uint4 l0 = make_uint4(0, 0, 0, 0), l1 = make_uint4(0, 0, 0, 0);
+        if (MODE) {
+          l0 = *reinterpret_cast<const uint4 *>(st + kPlaneBytes + off0);
+          l1 = *reinterpret_cast<const uint4 *>(st + kPlaneBytes + off1);
+        }
+        // activations of token gid, 32-column chunk 4g + tig, permuted even/odd
+        uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+        if (gid < M) {
+          const int c = g * 4 + tig;
+          xa = xs4[(gid * 2 + 0) * Cp + c];
+          xb = xs4[(gid * 2 + 1) * Cp + c];
+        }
+        // the accumulator starts at -offset * sum(q) of the group: the MMA
+        // result is the exact group sum of q * weight code
+        const int2 rr = *reinterpret_cast<const int2 *>(sr + g * 8 + tok0);
+        int d[4] = {-OFF * rr.x, -OFF * rr.y, -OFF * rr.x, -OFF * rr.y};
+        const uint32_t hw0[4] = {h0.x, h0.y, h0.z, h0.w}, hw1[4] = {h1.x, h1.y, h1.z, h1.w};
+        const uint32_t lw0[4] = {l0.x, l0.y, l0.z, l0.w}, lw1[4] = {l1.x, l1.y, l1.z, l1.w};
+        const uint32_t xe[4] = {xa.x, xa.z, xb.x, xb.z}, xo[4] = {xa.y, xa.w, xb.y, xb.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {  // 4 x K=32 columns of the group
+          uint32_t a[4];
+          if (MODE == 0) {
+            a[0] = hw0[jj] & 0x0F0F0F0Fu;
+            a[1] = hw1[jj] & 0x0F0F0F0Fu;
+            a[2] = (hw0[jj] >> 4) & 0x0F0F0F0Fu;
+            a[3] = (hw1[jj] >> 4) & 0x0F0F0F0Fu;
+          } else {
+            a[0] = ((hw0[jj] << 4) & 0xF0F0F0F0u) | (lw0[jj] & 0x0F0F0F0Fu);
+            a[1] = ((hw1[jj] << 4) & 0xF0F0F0F0u) | (lw1[jj] & 0x0F0F0F0Fu);
+            a[2] = (hw0[jj] & 0xF0F0F0F0u) | ((lw0[jj] >> 4) & 0x0F0F0F0Fu);
+            a[3] = (hw1[jj] & 0xF0F0F0F0u) | ((lw1[jj] >> 4) & 0x0F0F0F0Fu);
+          }
+          mma_u8s8(d, a, xe[jj], xo[jj], d);
+        }
+        if (DEBUG) {
+          const int n0 = row0 + r0, n1 = row0 + r1;
+          if (g < G) {
+            if (tok0 < M && n0 < p.N) p.S[((int64_t)tok0 * p.N + n0) * G + g] = d[0];
+            if (tok1 < M && n0 < p.N) p.S[((int64_t)tok1 * p.N + n0) * G + g] = d[1];
+            if (tok0 < M && n1 < p.N) p.S[((int64_t)tok0 * p.N + n1) * G + g] = d[2];
+            if (tok1 < M && n1 < p.N) p.S[((int64_t)tok1 * p.N + n1) * G + g] = d[3];
+          }
+        } else {
+          const float s0 = half_bits_to_float(q < 2 ? sc_cur0.x : sc_cur0.y, q & 1);
+          const float s1 = half_bits_to_float(q < 2 ? sc_cur1.x : sc_cur1.y, q & 1);
+          float x0 = 1.0f, x1 = 1.0f;
+          if (ACTG) {
+            const float2 xg = *reinterpret_cast<const float2 *>(sxg + g * 8 + tok0);
+            x0 = xg.x;
+            x1 = xg.y;
+          }
+          // |d| < 2^24: the conversions are exact
+          acc[0] = fmaf((float)d[0], ACTG ? s0 * x0 : s0, acc[0]);
+          acc[1] = fmaf((float)d[1], ACTG ? s0 * x1 : s0, acc[1]);
+          acc[2] = fmaf((float)d[2], ACTG ? s1 * x0 : s1, acc[2]);
+          acc[3] = fmaf((float)d[3], ACTG ? s1 * x1 : s1, acc[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (!DEBUG && ok) {
+      // every warp holds a K-slice of the same 16 x 8 outputs.  Each warp
+      // deposits its partial sums; the last warp to arrive adds the eight in
+      // a fixed warp order and writes y, so no warp waits at a CTA barrier.
+      const int slot = k % kRedSlots;
+      if (k >= kRedSlots) ok = mbar_wait_warp(&slot_free[slot], ((k / kRedSlots) - 1) & 1);
+      if (ok) {
+        float *rb = red + slot * (kConsumerWarps * 128);
+        *reinterpret_cast<float4 *>(rb + warp * 128 + lane * 4) =
+            make_float4(acc[0], acc[1], acc[2], acc[3]);
+        __threadfence_block();
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = atomicAdd(&cnt[slot], 1);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == kConsumerWarps - 1) {
+          __threadfence_block();
+          float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float4 pv = *reinterpret_cast<const float4 *>(rb + w * 128 + lane * 4);
+            v[0] += pv.x;
+            v[1] += pv.y;
+            v[2] += pv.z;
+            v[3] += pv.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tk = tok0 + (i & 1);
+            const int n = row0 + ((i >> 1) ? r1 : r0);
+            if (tk < M && n < p.N) {
+              float out = v[i];
+              if (!ACTG) out *= (i & 1) ? xt1 : xt0;
+              if (MODE) out *= 0.0625f;
+              if (p.bias) out += __half2float(__ushort_as_half(__ldg(p.bias + n)));
+              p.y[(int64_t)tk * p.N + n] = out;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) {
+            cnt[slot] = 0;
+            mbar_arrive(&slot_free[slot]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, uint64_t rows,
+              uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)esize};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int sms[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  return sms[dev] > 0 ? sms[dev] : 148;
+}
+
+// The plane as [segments of 128 bytes][rows][128 bytes]: a box of 16 rows x
+// 8 segments lands in shared memory as [segment][row][128 B] with the 128-byte
+// swizzle, the layout the MMA fragment loads read without bank conflicts.
+bool make_plane_map(CUtensorMap *m, const void *base, uint64_t N, uint64_t K) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, N, K / 256};
+  cuuint64_t strides[2] = {K / 2, 128};
+  cuuint32_t box[3] = {128, (cuuint32_t)kRows, (cuuint32_t)kSegs};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int M, bool ACTG, bool DEBUG>
+cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
+  Params p;
+  p.scale = a.scale;
+  p.xq = a.xq;
+  p.xscale = a.xscale;
+  p.xsum = a.xsum;
+  p.bias = a.bias;
+  p.y = a.y;
+  p.S = a.S;
+  p.M = (int)a.M;
+  p.N = (int)a.N;
+  p.K = (int)a.K;
+  p.G = (int)(a.K / kGroup);
+  p.nks = (int)((a.K + kStepCols - 1) / kStepCols);
+  p.Cp = p.nks * (kStepCols / 32);
+  p.Gp = p.nks * (kStepCols / kGroup);
+  p.NB = (int)((a.N + kRows - 1) / kRows);
+  // balanced grid: every CTA gets ceil(NB / grid) or one fewer 16-row blocks
+  const int sms = num_sms();
+  const int per = (p.NB + sms - 1) / sms;
+  const int grid = (p.NB + per - 1) / per;
+  const int fixed = smem_total(MODE, M, ACTG, p.K, per, 0);
+  int stages = (kSmemBudget - fixed) / stage_bytes(MODE);
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) return cudaErrorInvalidValue;
+  p.stages = stages;
+  const int smem = smem_total(MODE, M, ACTG, p.K, per, stages);
+
+  CUtensorMap mh, ml;
+  if (!make_plane_map(&mh, a.hi, (uint64_t)a.N, (uint64_t)a.K)) return cudaErrorInvalidValue;
+  ml = mh;
+  if (MODE && !make_plane_map(&ml, a.lo, (uint64_t)a.N, (uint64_t)a.K)) return cudaErrorInvalidValue;
+
+  auto kern = gemv_tma_kernel<MODE, M, ACTG, DEBUG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, a.overlap, mh, ml,
+                 p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int MODE, bool DEBUG>
+cudaError_t dispatch_m(const LinearArgs &a, cudaStream_t st) {
+  const bool g = a.act_group != 0 && !DEBUG;
+#define BITNEST_GV_CASE(MM) \
+  case MM: return g ? launch_t<MODE, MM, true, DEBUG>(a, st) : launch_t<MODE, MM, false, DEBUG>(a, st);
+  switch (a.M) {
+    BITNEST_GV_CASE(1)
+    BITNEST_GV_CASE(2)
+    BITNEST_GV_CASE(3)
+    BITNEST_GV_CASE(4)
+    BITNEST_GV_CASE(5)
+    BITNEST_GV_CASE(6)
+    BITNEST_GV_CASE(7)
+    BITNEST_GV_CASE(8)
+    default: return cudaErrorInvalidValue;
+  }
+#undef BITNEST_GV_CASE
+}
+
+}  // namespace gv
+
+bool gemv_tma_supported(int64_t M, int64_t N, int64_t K) {
+  // the scale rows are read as 32-bit words and G is a multiple of 8
+  if (M < 1 || M > 8 || N < 1 || K % 1024 != 0 || K > (1 << 20)) return false;
+  const int64_t NB = (N + gv::kRows - 1) / gv::kRows;
+  const int sms = gv::num_sms();
+  const int64_t per = (NB + sms - 1) / sms;
+  const int G = (int)(K / kGroup);
+  if (per * gv::kRows * gv::scale_pitch(G) * 2 > gv::kScaleSmemMax) return false;
+  return gv::smem_total(1, (int)M, true, (int)K, (int)per, 2) <= gv::kSmemBudget;
+}
+
+cudaError_t launch_gemv_tma(const LinearArgs &a, cudaStream_t st) {
+  const bool debug = a.S != nullptr;
+  if (a.mode == 0) return debug ? gv::dispatch_m<0, true>(a, st) : gv::dispatch_m<0, false>(a, st);
+  return debug ? gv::dispatch_m<1, true>(a, st) : gv::dispatch_m<1, false>(a, st);
+}
+
+cudaError_t read_wait_timeout_gemv(int *flag, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(flag, g_wait_timeout, sizeof(int));
+  if (e != cudaSuccess || !reset) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_wait_timeout, &zero, sizeof(int));
+}
+
+}  // namespace bitnest

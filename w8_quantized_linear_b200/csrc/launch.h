@@ -19,6 +19,7 @@ struct LinearArgs {
   int32_t *S;             // debug group sums [M, N, K/128] (null unless debug)
   int64_t M, N, K;
   int act_group;          // 0 or 128
+  bool overlap;           // launch with programmatic dependent launch
 };
 
 cudaError_t launch_pack(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K, uint8_t *hi,
@@ -31,6 +32,11 @@ cudaError_t launch_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_
 // Largest M * K the GEMV kernels can stage in shared memory.
 bool gemv_fits(int64_t M, int64_t K);
 cudaError_t launch_gemv(const LinearArgs &a, cudaStream_t st);
+
+// TMA-ring decode GEMV (K a multiple of 1024).
+bool gemv_tma_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemv_tma(const LinearArgs &a, cudaStream_t st);
+cudaError_t read_wait_timeout_gemv(int *flag, bool reset);
 
 // tcgen05 tensor-core GEMM (any M).
 bool tc_supported(int64_t M, int64_t N, int64_t K);

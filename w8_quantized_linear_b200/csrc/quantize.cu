@@ -74,6 +74,10 @@ __global__ void __launch_bounds__(T) quantize_token_kernel(const uint16_t *__res
                                                            int64_t K, int8_t *__restrict__ xq,
                                                            float *__restrict__ xs,
                                                            int32_t *__restrict__ xsum) {
+  // x may come from the preceding kernel: wait for it, and only then let the
+  // next kernel (the layer, which may stream its weights early) start
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t m = blockIdx.x;
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + m * K);
   const int nvec = (int)(K / 8);
@@ -108,6 +112,8 @@ __global__ void __launch_bounds__(256) quantize_group_kernel(const uint16_t *__r
                                                              int8_t *__restrict__ xq,
                                                              float *__restrict__ xs,
                                                              int32_t *__restrict__ xsum) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t nvec = M * K / 8;
   const int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // vectors in order
   const bool ok = v < nvec;  // nvec is a multiple of 16: whole groups share `ok`
@@ -132,14 +138,18 @@ __global__ void __launch_bounds__(256) quantize_group_kernel(const uint16_t *__r
 
 cudaError_t launch_quantize(const uint16_t *x, int64_t M, int64_t K, int act_group, int8_t *xq,
                             float *xs, int32_t *xsum, cudaStream_t st) {
+  // programmatic dependent launch: the kernel waits for its predecessor first
+  cudaError_t e;
   if (act_group == 0) {
-    quantize_token_kernel<512><<<(unsigned)M, 512, 0, st>>>(x, K, xq, xs, xsum);
+    e = launch_pdl(quantize_token_kernel<512>, dim3((unsigned)M), dim3(512), 0, st, true, x, K, xq,
+                   xs, xsum);
   } else {
     const int64_t nvec = M * K / 8;
     const int threads = 256;
-    quantize_group_kernel<<<(unsigned)((nvec + threads - 1) / threads), threads, 0, st>>>(
-        x, M, K, xq, xs, xsum);
+    e = launch_pdl(quantize_group_kernel, dim3((unsigned)((nvec + threads - 1) / threads)),
+                   dim3(threads), 0, st, true, x, M, K, xq, xs, xsum);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
