@@ -22,8 +22,9 @@
 // keep up with HBM at 2 warps per scheduler.  The K-permutation that lets a
 // plane word's low / high nibbles feed the fragments without byte shuffles is
 // applied to the staged activations instead (even / odd columns).  Each warp
-// accumulates its groups' scaled sums in fp32; the 8 warps' partial sums of a
-// 16-row block are added in a fixed order by the last warp to finish it.
+// accumulates its groups' scaled sums in fp32 and hands the partial sums of a
+// 16-row block to a reducer warp, which adds them in a fixed warp order and
+// writes y while the consumers go on with the next block.
 //
 // With programmatic dependent launch the weight stream starts while the
 // preceding kernel (the activation quantiser) still runs; the consumers wait
@@ -40,13 +41,15 @@ namespace gv {
 
 constexpr int kConsumerWarps = 8;                      // four 128-column groups each per stage
 constexpr int kGroupsPerWarp = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;    // + one producer warp
+constexpr int kProducerWarp = kConsumerWarps;          // TMA producer
+constexpr int kReducerWarp = kConsumerWarps + 1;       // adds the warps' partial sums, writes y
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kRows = 16;                              // weight rows per stage (the MMA's M)
 constexpr int kStepCols = 4096;                        // columns per stage = 32 groups
 constexpr int kSegs = kStepCols / 256;                 // 128-byte plane segments per row
 constexpr int kPlaneBytes = kRows * kStepCols / 2;     // 32 KB: one TMA box per plane
 constexpr int kMaxStages = 8;
-constexpr int kRedSlots = 2;  // row blocks whose partial sums can be in flight
+constexpr int kRedSlots = 4;  // row blocks whose partial sums can be in flight
 constexpr int kScaleSmemMax = 32 * 1024;  // the CTA's group scales are staged once
 constexpr int kSmemBudget = 227 * 1024;
 
@@ -76,13 +79,13 @@ __host__ __device__ inline int fixed_bytes(int M, int K, bool actg, int nb) {
   const int Cp = nks * (kStepCols / 32), Gp = nks * (kStepCols / kGroup);
   const int G = K / kGroup;
   int o = M * Cp * 32 + Gp * 32 + (actg ? Gp * 32 : 0) + (nb * kRows * scale_pitch(G) * 2 + 15) / 16 * 16 +
-          kRedSlots * kConsumerWarps * 128 * 4 + kRedSlots * 4;
+          kRedSlots * kConsumerWarps * 128 * 4;
   return (o + 1023) / 1024 * 1024;
 }
 
 __host__ inline int smem_total(int mode, int M, bool actg, int K, int nb, int stages) {
   return 1024 + fixed_bytes(M, K, actg, nb) + stages * stage_bytes(mode) +
-         (2 * kMaxStages + kRedSlots) * 8;
+         (2 * kMaxStages + 2 * kRedSlots) * 8;
 }
 
 // D = A (16x32 u8) * B (32x8 s8) + C, int32.  Not volatile: a pure function
@@ -145,11 +148,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __half *ssc = reinterpret_cast<__half *>(sxg + (ACTG ? Gp * 8 : 0));  // [nb * 16][sp]
   float *red = reinterpret_cast<float *>(
       reinterpret_cast<uint8_t *>(ssc) + (nb * kRows * sp * 2 + 15) / 16 * 16);  // [slots][warps][128]
-  int *cnt = reinterpret_cast<int *>(red + kRedSlots * kConsumerWarps * 128);  // [slots]
   uint8_t *ring = smem + fixed_bytes(M, p.K, ACTG, nb);            // 1024-aligned stages
   uint64_t *full = reinterpret_cast<uint64_t *>(ring + S * STAGE);
   uint64_t *empty = full + kMaxStages;
-  uint64_t *slot_free = empty + kMaxStages;  // [kRedSlots]: partial-sum slot read out
+  uint64_t *part_full = empty + kMaxStages;       // [kRedSlots]: all warps' partials written
+  uint64_t *slot_free = part_full + kRedSlots;    // [kRedSlots]: partials read out
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -159,15 +162,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], kConsumerWarps);
     }
     for (int i = 0; i < kRedSlots; ++i) {
+      mbar_init(&part_full[i], kConsumerWarps);
       mbar_init(&slot_free[i], 1);
-      cnt[i] = 0;
     }
     fence_barrier_init();
   }
   __syncthreads();
   griddep_launch_dependents();
 
-  if (warp == kConsumerWarps) {
+  if (warp == kReducerWarp) {
+    // ------------------------------------------------------------- reducer
+    // every consumer warp holds a K-slice of the same 16 x 8 outputs of a
+    // row block; add the eight in a fixed warp order and write y
+    if (DEBUG) return;
+    griddep_wait();  // the token scales come from the preceding kernel
+    const int gid = lane >> 2, tig = lane & 3;
+    const int r0 = perm_row(gid), r1 = r0 + 8;
+    const int t0 = 2 * tig;
+    float xt0 = 0.0f, xt1 = 0.0f;
+    if (!ACTG) {
+      xt0 = t0 < M ? __ldg(p.xscale + t0) : 0.0f;
+      xt1 = t0 + 1 < M ? __ldg(p.xscale + t0 + 1) : 0.0f;
+    }
+    for (int k = 0; k < nb; ++k) {
+      const int slot = k % kRedSlots;
+      if (!mbar_wait_warp(&part_full[slot], (k / kRedSlots) & 1)) return;
+      const float *rb = red + slot * (kConsumerWarps * 128);
+      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float4 pv = *reinterpret_cast<const float4 *>(rb + w * 128 + lane * 4);
+        v[0] += pv.x;
+        v[1] += pv.y;
+        v[2] += pv.z;
+        v[3] += pv.w;
+      }
+      const int row0 = ((int)blockIdx.x + k * (int)gridDim.x) * kRows;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tk = t0 + (i & 1);
+        const int n = row0 + ((i >> 1) ? r1 : r0);
+        if (tk < M && n < p.N) {
+          float out = v[i];
+          if (!ACTG) out *= (i & 1) ? xt1 : xt0;
+          if (MODE) out *= 0.0625f;
+          if (p.bias) out += __half2float(__ushort_as_half(__ldg(p.bias + n)));
+          p.y[(int64_t)tk * p.N + n] = out;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&slot_free[slot]);
+    }
+    return;
+  }
+
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_hi);
@@ -213,13 +262,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   griddep_wait();  // the activations are written by the preceding kernel
   const int C = p.K / 32;
-  // activations: every load of this thread first, then the permuted stores
-  constexpr int XB = 8;  // items per batch
-  for (int base = threadIdx.x; base < M * Cp; base += XB * NT) {
+  // activations and group sums: every load of this thread first (one round
+  // trip), then the permuted stores
+  constexpr int XB = 8;  // activation items per batch
+  constexpr int RB = 4;  // group-sum items per batch
+  for (int bx = 0, br = 0; bx < M * Cp || br < Gp * 8; bx += XB * NT, br += RB * NT) {
     uint4 va[XB], vb[XB];
+    int rv[RB];
+    float xv[RB];
 #pragma unroll
     for (int u = 0; u < XB; ++u) {
-      const int item = base + u * NT;
+      const int item = bx + threadIdx.x + u * NT;
       va[u] = make_uint4(0, 0, 0, 0);
       vb[u] = make_uint4(0, 0, 0, 0);
       if (item < M * Cp) {
@@ -232,8 +285,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 #pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      const int i = br + threadIdx.x + u * NT;
+      const int g = i >> 3, m = i & 7;
+      const bool in = i < Gp * 8 && m < M && g < G;
+      rv[u] = in ? __ldg(p.xsum + m * G + g) : 0;
+      xv[u] = (ACTG && in) ? __ldg(p.xscale + m * G + g) : 0.0f;
+    }
+#pragma unroll
     for (int u = 0; u < XB; ++u) {
-      const int item = base + u * NT;
+      const int item = bx + threadIdx.x + u * NT;
       if (item < M * Cp) {
         const int m = item / Cp, c = item - m * Cp;
         const uint32_t w[8] = {va[u].x, va[u].y, va[u].z, va[u].w,
@@ -248,33 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         xs4[(m * 2 + 1) * Cp + c] = make_uint4(e[2], o[2], e[3], o[3]);
       }
     }
-  }
-  // group sums (and per-group activation scales), [Gp][8]
-  for (int base = threadIdx.x; base < Gp * 8; base += 4 * NT) {
-    int rv[4];
-    float xv[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = base + u * NT;
-      const int g = i >> 3, m = i & 7;
-      const bool in = i < Gp * 8 && m < M && g < G;
-      rv[u] = in ? __ldg(p.xsum + m * G + g) : 0;
-      xv[u] = (ACTG && in) ? __ldg(p.xscale + m * G + g) : 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = base + u * NT;
+    for (int u = 0; u < RB; ++u) {
+      const int i = br + threadIdx.x + u * NT;
       if (i < Gp * 8) {
         sr[i] = rv[u];
         if (ACTG) sxg[i] = xv[u];
       }
     }
-  }
-  float xt0 = 0.0f, xt1 = 0.0f;  // token scales of this thread's two output columns
-  if (!ACTG && !DEBUG) {
-    const int t0 = 2 * (lane & 3);
-    xt0 = t0 < M ? __ldg(p.xscale + t0) : 0.0f;
-    xt1 = t0 + 1 < M ? __ldg(p.xscale + t0 + 1) : 0.0f;
   }
   cp_async_wait_all();
   asm volatile("bar.sync 1, %0;" ::"r"(NT) : "memory");
@@ -378,49 +420,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&empty[s]);
     }
     if (!DEBUG && ok) {
-      // every warp holds a K-slice of the same 16 x 8 outputs.  Each warp
-      // deposits its partial sums; the last warp to arrive adds the eight in
-      // a fixed warp order and writes y, so no warp waits at a CTA barrier.
+      // deposit this warp's partial sums of the row block for the reducer
       const int slot = k % kRedSlots;
       if (k >= kRedSlots) ok = mbar_wait_warp(&slot_free[slot], ((k / kRedSlots) - 1) & 1);
       if (ok) {
         float *rb = red + slot * (kConsumerWarps * 128);
         *reinterpret_cast<float4 *>(rb + warp * 128 + lane * 4) =
             make_float4(acc[0], acc[1], acc[2], acc[3]);
-        __threadfence_block();
         __syncwarp();
-        int prev = 0;
-        if (lane == 0) prev = atomicAdd(&cnt[slot], 1);
-        prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev == kConsumerWarps - 1) {
-          __threadfence_block();
-          float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) {
-            const float4 pv = *reinterpret_cast<const float4 *>(rb + w * 128 + lane * 4);
-            v[0] += pv.x;
-            v[1] += pv.y;
-            v[2] += pv.z;
-            v[3] += pv.w;
-          }
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int tk = tok0 + (i & 1);
-            const int n = row0 + ((i >> 1) ? r1 : r0);
-            if (tk < M && n < p.N) {
-              float out = v[i];
-              if (!ACTG) out *= (i & 1) ? xt1 : xt0;
-              if (MODE) out *= 0.0625f;
-              if (p.bias) out += __half2float(__ushort_as_half(__ldg(p.bias + n)));
-              p.y[(int64_t)tk * p.N + n] = out;
-            }
-          }
-          __syncwarp();
-          if (lane == 0) {
-            cnt[slot] = 0;
-            mbar_arrive(&slot_free[slot]);
-          }
-        }
+        if (lane == 0) mbar_arrive(&part_full[slot]);
       }
     }
   }
