@@ -245,10 +245,11 @@ class DecodeWorkload:
     def _path(self):
         return self.bn.PATH_AUTO | (self.bn.PATH_OVERLAP if self.overlap else 0)
 
-    def run_step(self, copy, events=None, e2e=False):
+    def run_step(self, copy, events=None, e2e=False, qevents=None):
         """Enqueue one step on the current stream: the draft pass then the
         verify pass, each quantise + linear for the four layer groups.
-        `events`: per (group, mode) (start, end) CUDA events around the linear."""
+        `events` / `qevents`: per (group, mode) (start, end) CUDA events around
+        the linear / the quantiser."""
         bn = self.bn
         w = self.copies[copy]
         for mode in (0, 1):
@@ -258,7 +259,11 @@ class DecodeWorkload:
                 x = self.x[gname, mode]
                 if e2e:
                     x.copy_(self.x_host[gname, mode], non_blocking=True)
+                if qevents is not None:
+                    qevents[gname, mode][0].record()
                 bn.quantize_act(x, g, out=(b["xq"], b["xs"], b["xsum"]))
+                if qevents is not None:
+                    qevents[gname, mode][1].record()
                 hi, lo, s = w[gname]
                 if events is not None:
                     events[gname, mode][0].record()
@@ -431,9 +436,13 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
     # time from CUDA events recorded on the launching stream right around each
     # launch; a spin kernel first lets the host enqueue the whole sequence, so
     # no launch waits on the host between its two events.
-    events = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for k in wl.bufs}
+    def ev_pairs():
+        return {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for k in wl.bufs}
+
+    events, qevents = ev_pairs(), ev_pairs()
     dur = {k: 0.0 for k in events}
+    qdur = {k: 0.0 for k in events}
     n_ev = max(8, min(args.steps, 200))
     for i in range(n_ev):
         torch.cuda._sleep(4_000_000)
@@ -441,17 +450,28 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
         torch.cuda.synchronize()
         for k, (a, b) in events.items():
             dur[k] += a.elapsed_time(b) / 1e3
+    # the quantisers on their own pass (no events between them and their linear)
+    for i in range(n_ev):
+        torch.cuda._sleep(4_000_000)
+        wl.run_step(i % N_COPIES, qevents=qevents)
+        torch.cuda.synchronize()
+        for k, (a, b) in qevents.items():
+            qdur[k] += a.elapsed_time(b) / 1e3
     per_group = {}
     for (gname, mode) in events:
         N, K, _ = group_shape(dict(LAYER_GROUPS)[gname])
         d = dur[gname, mode] / n_ev
         b = linear_bytes(mode, DECODE_M[mode], N, K)
+        _, _, g = group_shape(dict(LAYER_GROUPS)[gname])
+        dq = qdur[gname, mode] / n_ev
         per_group[f"{gname}/{'draft' if mode == 0 else 'target'}"] = {
             "N": N, "K": K, "us": round(d * 1e6, 3), "GB/s": round(b / d / 1e9, 1),
-            "frac_hbm": round(b / d / 1e9 / hbm_peak, 3)}
+            "frac_hbm": round(b / d / 1e9 / hbm_peak, 3),
+            "quantise_us": round(dq * 1e6, 3),
+            "quantise_GB/s": round(quant_bytes(DECODE_M[mode], K, g) / dq / 1e9, 1)}
     # the dominant launch: the fused gate|up verify (target, M = 4) linear
-    N, K, _ = group_shape(dict(LAYER_GROUPS)["gate_up"])
-    dom_bytes = linear_bytes(1, DECODE_M[1], N, K)
+    dom_N, dom_K, _ = group_shape(dict(LAYER_GROUPS)["gate_up"])
+    dom_bytes = linear_bytes(1, DECODE_M[1], dom_N, dom_K)
     dom_time = dur["gate_up", 1] / n_ev
     achieved = dom_bytes / dom_time / 1e9
     # every projection on its own (unfused), same events
@@ -476,7 +496,7 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
                 "frac_hbm": round(b / t / 1e9 / hbm_peak, 3)}
     roofline = {
         "bound": "hbm",
-        "kernel": f"gemv_tma_kernel<TARGET, M=4>, fused gate|up (N={N}, K={K})",
+        "kernel": f"gemv_tma_kernel<TARGET, M=4>, fused gate|up (N={dom_N}, K={dom_K})",
         "achieved": round(achieved, 1),
         "peak": hbm_peak,
         "unit": "GB/s",
@@ -493,6 +513,129 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
 
 
 
+# ------------------------------------------------------------- M sweep
+SWEEP_M = (1, 2, 4, 8, 16, 32, 64, 128)
+SWEEP_SHAPES = ("gate_proj", "down_proj")  # 14336 x 4096 and 4096 x 14336
+
+
+def measure_sweep(wl, hbm_peak, reps=5):
+    """Every M of the batch / verify sweep on the two MLP shapes, both modes:
+    the path the library picks, device time per launch (CUDA events around the
+    launch, after a 256 MB L2 flush), HBM throughput and int8 TOPS."""
+    import torch
+
+    bn = wl.bn
+    dev = wl.dev
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    res = {}
+    torch.cuda._sleep(200_000_000)  # about 0.1 s of spinning: clocks up before the first case
+    torch.cuda.synchronize()
+    for name in SWEEP_SHAPES:
+        N, K, g = synth.LLAMA3_8B_PROJECTIONS[name]
+        hi, lo, sc = wl.single[name]
+        pid = synth.PROJ_IDS[name]
+        for M in SWEEP_M:
+            x = torch.from_numpy(synth.activations(synth.SEED_ACTS + pid + 1000 * M, M, K)).to(dev)
+            xq, xs, xsum = bn.quantize_act(x, g)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            for mode in (0, 1):
+                path = bn.select_path(mode, M, N, K)
+                bn.linear(mode, hi, lo, sc, xq, xs, xsum, g, out=y)  # warm
+                t = 0.0
+                for _ in range(reps):
+                    flush.fill_(1)
+                    a.record()
+                    bn.linear(mode, hi, lo, sc, xq, xs, xsum, g, out=y)
+                    b.record()
+                    torch.cuda.synchronize()
+                    t += a.elapsed_time(b) / 1e3
+                t /= reps
+                nb = linear_bytes(mode, M, N, K)
+                res[f"{name}/{'draft' if mode == 0 else 'target'}/M={M}"] = {
+                    "path": "gemv" if path == bn.PATH_GEMV else "tcgen05",
+                    "us": round(t * 1e6, 2), "GB/s": round(nb / t / 1e9, 1),
+                    "frac_hbm": round(nb / t / 1e9 / hbm_peak, 3),
+                    "TOPS": round(2.0 * M * N * K / t / 1e12, 2)}
+            del x, xq, xs, xsum, y
+    del flush
+    return res
+
+
+# --------------------------------------------------------- decode round
+ROUND_LAYERS = 32
+ROUND_DRAFT_PASSES = 3  # gamma = 3 draft tokens, then one verify pass at M = gamma + 1
+
+
+def round_bytes():
+    """Algorithmic bytes of one speculative decode round over the 32 layers."""
+    per = {}
+    for mode, M in DECODE_M.items():
+        per[mode] = sum(linear_bytes(mode, M, *group_shape(m)[:2]) + quant_bytes(M, *group_shape(m)[1:])
+                        for _, m in LAYER_GROUPS)
+    return ROUND_LAYERS * (ROUND_DRAFT_PASSES * per[0] + per[1])
+
+
+def measure_round(wl, hbm_peak, reps=10):
+    """One speculative decode round on 32 layers of Llama-3-8B-shaped nested
+    weights (3.5 GB hi + 3.5 GB lo planes): three draft passes at M = 1, then
+    the verify pass at M = 4, every layer's four quantise + linear pairs, as
+    one CUDA graph.  The layer weights are drawn on the device by torch's
+    seeded generator (uniform plane bytes = uniform nibbles; scales
+    1e-4 + 0.005 |N(0,1)| in fp16); they are only timed, never checked."""
+    import torch
+
+    bn = wl.bn
+    dev = wl.dev
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6000)
+    layers = []
+    for _ in range(ROUND_LAYERS):
+        lw = {}
+        for gname, members in LAYER_GROUPS:
+            N, K, _ = group_shape(members)
+            hi = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=gen)
+            lo = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=gen)
+            z = torch.randn((N, K // 128), device=dev, generator=gen)
+            lw[gname] = (hi, lo, (1e-4 + 0.005 * z.abs()).half())
+        layers.append(lw)
+    path = bn.PATH_AUTO | (bn.PATH_OVERLAP if wl.overlap else 0)
+
+    def one_round():
+        for p in range(ROUND_DRAFT_PASSES + 1):
+            mode = 1 if p == ROUND_DRAFT_PASSES else 0
+            for lw in layers:
+                for gname, members in LAYER_GROUPS:
+                    _, _, g = group_shape(members)
+                    b = wl.bufs[gname, mode]
+                    bn.quantize_act(wl.x[gname, mode], g, out=(b["xq"], b["xs"], b["xsum"]))
+                    hi, lo, s = lw[gname]
+                    bn.linear(mode, hi, lo, s, b["xq"], b["xs"], b["xsum"], g, out=b["y"], path=path)
+
+    graph = capture(one_round)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    t = timed_replays([graph], reps, lambda: None) / reps
+    graph.reset()
+    del layers
+    torch.cuda.empty_cache()
+    nb = round_bytes()
+    launches = (ROUND_DRAFT_PASSES + 1) * ROUND_LAYERS * len(LAYER_GROUPS) * 2
+    return {
+        "workload": "speculative round: 32 layers x 7 projections, 3 draft passes (M=1) + "
+                    "1 verify pass (M=4), quantisers included, one CUDA graph",
+        "us_per_round": round(t * 1e6, 1),
+        "GB_per_round": round(nb / 1e9, 3),
+        "GB_per_token_full_acceptance": round(nb / 1e9 / (ROUND_DRAFT_PASSES + 1), 3),
+        "GB/s": round(nb / t / 1e9, 1),
+        "frac_hbm": round(nb / t / 1e9 / hbm_peak, 3),
+        "launches_per_round": launches,
+        "rounds_timed": reps,
+    }
+
+
 # ------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -507,9 +650,10 @@ def main():
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step's kernels directly instead of replaying a CUDA graph "
                          "(for profilers that cannot replay the captured kernel nodes)")
-    ap.add_argument("--workload", default="all", choices=["all", "decode", "prefill"],
-                    help="all: the decode step line with the prefill object; decode / "
-                         "prefill: only that part (for profiling runs)")
+    ap.add_argument("--workload", default="all",
+                    choices=["all", "decode", "prefill", "sweep", "round"],
+                    help="all: the decode step line with the prefill, M-sweep and "
+                         "decode-round objects; otherwise only that part (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -552,6 +696,11 @@ def main():
     dec = None
     if args.workload in ("all", "decode"):
         dec = measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind)
+    sweep = rnd = None
+    if args.workload in ("all", "sweep"):
+        sweep = measure_sweep(wl, hbm_peak, reps=5 if args.workload == "all" else 2)
+    if args.workload in ("all", "round"):
+        rnd = measure_round(wl, hbm_peak, reps=10 if args.workload == "all" else 3)
     prefill = None
     if args.workload in ("all", "prefill"):
         pre, pre_ops, pre_t = measure_prefill(wl, reps=10 if args.workload == "all" else 3)
@@ -572,8 +721,9 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "workload": "prefill only", "prefill": prefill}),
-                  flush=True)
+            part = {"prefill": prefill, "m_sweep": sweep, "decode_round": rnd}
+            print(json.dumps({"metric": METRIC, "workload": f"{args.workload} only",
+                              **{k: v for k, v in part.items() if v is not None}}), flush=True)
         return
     value, ms_per_step, clocks, e2e_value, h2d, d2h, roofline = dec
 
@@ -613,6 +763,12 @@ def main():
     }
     if prefill is not None:
         out["prefill"] = prefill
+    if sweep is not None:
+        out["m_sweep"] = {"workload": "M in {1..128} x gate_proj 14336x4096 / down_proj "
+                                      "4096x14336 x draft / target, one launch after an L2 flush",
+                          "per_case": sweep}
+    if rnd is not None:
+        out["decode_round"] = rnd
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, cores, rows = cpu_baseline()
         out["cpu_baseline"] = {
