@@ -355,7 +355,7 @@ def measure_prefill(wl, reps=10):
         x = torch.from_numpy(synth.activations(synth.SEED_ACTS + pid, PREFILL_M, K)).to(dev)
         xq, xs, xsum = bn.quantize_act(x, g)
         y = torch.empty((PREFILL_M, N), dtype=torch.float32, device=dev)
-        hi, lo, sc = wl.copies[0][name]
+        hi, lo, sc = wl.single[name]
         bn.linear(1, hi, lo, sc, xq, xs, xsum, g, out=y)  # warm
         t = 0.0
         for _ in range(reps):

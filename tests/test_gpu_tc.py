@@ -107,3 +107,18 @@ def test_llama3_prefill_sampled(name):
     S_ref = oracle.group_sums(1, oracle.pack_plane(uh[:256]), oracle.pack_plane(ul[:256]),
                               q[toks], K)
     assert np.array_equal(S[toks], S_ref)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("act_group", [0, 128])
+def test_tc_persistent_tiles(mode, act_group):
+    """More tiles (32 row tiles x 5 token tiles, both ragged) than SMs: every
+    CTA walks several tiles; outputs and exact sums over the whole problem."""
+    M, N, K = 600, 4000, 256
+    p = Problem(M, N, K, seed=77 + mode, act_group=act_group)
+    y = p.y_gpu(mode, path=bn.PATH_TC)
+    assert oracle.max_normalised_error(y, p.y_ref(mode)) <= TOL
+    if act_group == 0:
+        S = bn.debug_group_sums(mode, p.d_hi, p.d_lo, p.d_xq, p.d_xsum, path=bn.PATH_TC)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(S), oracle.group_sums(mode, p.hi, p.lo, p.q, K))

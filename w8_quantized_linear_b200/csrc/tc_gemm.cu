@@ -1,25 +1,34 @@
-// tcgen05 tensor-core path of the bit-nested linear layer (any M).
+// tcgen05 tensor-core path of the bit-nested linear layer (any M; the
+// prefill-sized GEMM and the middle of the batch sweep).
 //
 // BitNest-Llama-3-8B model card, section "Files": the draft weight code is
 // hi - 8 and the target code 16 (hi - 8) + (lo - 8) = ((hi << 4) | lo) - 136.
 // Both are formed here as ONE unsigned byte per weight (hi, or (hi<<4)|lo)
 // so a single kind::i8 MMA (u8 weights x s8 activations -> s32) per 32
 // columns does the work; the constant offset (8 or 136) times the
-// activation group sum is folded into the epilogue.
+// activation group sum is folded into the drain.
 //
 // Tile: 128 weight rows (the MMA's M, TMEM lanes) x BT tokens (the MMA's N),
 // one 128-column group per pipeline stage.  The group scales differ per
 // (row, group), so the int32 accumulator of every group is drained from TMEM
-// and scaled in fp32; two TMEM accumulators let the drain of group g overlap
-// the MMA of group g + 1.
+// and scaled in fp32 (the model card's per-group scale); four TMEM
+// accumulators let the drain of a group run while the MMAs of the next
+// three proceed.  Persistent: one CTA per SM walks the tiles (token tiles
+// fastest, so the CTAs of a wave share weight rows in L2) and every role
+// runs ahead into the next tile while the epilogue finishes the current one.
+//
+// Every input stream runs well ahead of the MMAs: the TMA ring carries the
+// activation tile and the plane tiles of a group per stage, and the
+// per-group constants (row scales, per-token offsets) are read eight groups
+// per round trip into a ring of their own.
 //
 // Warp roles (15 warps):
-//   0      TMA producer: activation tile (128-byte swizzle) and the hi / lo
+//   0..3   plane -> byte operand (shared-memory planes -> swizzled K-major)
+//   4      TMA producer: activation tile (128-byte swizzle) and the hi / lo
 //          plane tiles of the group, one mbarrier per stage (no multicast)
-//   1      TMEM owner and MMA issuer (one thread)
-//   2      per-group column constants: magic - offset * activation group sum
-//          (and the per-group activation scale for o_proj-style inputs)
-//   3..6   plane -> byte transform into the swizzled K-major MMA operand
+//   5      TMEM owner and MMA issuer (one thread)
+//   6      per-group constants: row scales, magic - offset * activation group
+//          sum per token (and the per-group activation scale for o_proj)
 //   7..14  epilogue: TMEM -> registers, exact int -> fp32, scale, accumulate
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -33,9 +42,12 @@ namespace bitnest {
 namespace tc {
 
 constexpr int BW = 128;  // weight rows per tile
-constexpr int kMaxStages = 4;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpPrep = 2;
-constexpr int kWarpXf0 = 3, kNumXf = 4;
+constexpr int kMaxStages = 8;
+constexpr int kAccBufs = 4;    // TMEM accumulators
+constexpr int kCSlots = 16;    // per-group constant slots
+constexpr int kCBatch = 8;     // groups of constants per round trip
+constexpr int kWarpXf0 = 0, kNumXf = 4;
+constexpr int kWarpTma = 4, kWarpMma = 5, kWarpPrep = 6;
 constexpr int kWarpEpi0 = 7, kNumEpi = 8;
 constexpr int kWarps = 15;
 constexpr int kThreads = kWarps * 32;
@@ -51,91 +63,103 @@ struct Params {
   const uint16_t *bias;    // [N] or null
   float *y;                // [M, N]
   int32_t *S;              // debug sums [M, N, G]
-  int M, N, G;
-  int act_group;
+  int M, N, K, G;
+  int mt;                  // token tiles
+  int tiles;               // row tiles x token tiles
   int stages;
-  int sc_pitch;            // halves per row of the staged scale block (odd word count)
 };
 
 __host__ __device__ constexpr int tmem_cols(int bt) {
-  return 2 * bt < 32 ? 32 : 2 * bt;  // 2 * bt is a power of two for bt in {16,32,64,128}
+  // kAccBufs * bt rounded up to a power of two >= 32
+  return kAccBufs * bt <= 32 ? 32 : kAccBufs * bt <= 64 ? 64 : kAccBufs * bt <= 128 ? 128
+         : kAccBufs * bt <= 256 ? 256 : 512;
 }
 
-struct Layout {
-  int a, b, h, l, sc, cv, xv, bars, total;
-};
-
-__host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
-
-__host__ __device__ inline Layout smem_layout(int mode, int bt, int stages, int G, int pitch) {
-  Layout L;
-  int o = 0;
-  L.a = o;
-  o += stages * BW * 128;
-  L.b = o;
-  o += stages * bt * 128;
-  L.h = o;
-  o += stages * BW * 64;
-  L.l = o;
-  o += mode ? stages * BW * 64 : 0;
-  L.sc = o;
-  o += align_up(BW * pitch * 2, 16);
-  L.cv = o;
-  o += stages * bt * 4;
-  L.xv = o;
-  o += stages * bt * 4;
-  o = align_up(o, 8);
-  L.bars = o;
-  o += (5 * kMaxStages + 4) * 8 + 16;
-  L.total = o + 1024;  // slack to align the base to 1024 bytes
-  return L;
+__host__ __device__ constexpr int stage_bytes(int mode, int bt) {
+  // operand A (128 x 128 B), operand B (bt x 128 B), hi (and lo) plane tiles
+  // (128 x 64 B each); stages start on 1024-byte boundaries (the 128-byte
+  // swizzle atom)
+  return (BW * 128 + bt * 128 + (mode ? 2 : 1) * BW * 64 + 1023) / 1024 * 1024;
 }
 
-template <int MODE, int BT, bool DEBUG>
+// one constant slot: row scales (128 fp32), column constants and activation
+// scales (bt x 4 B each)
+__host__ __device__ constexpr int cslot_bytes(int bt) { return BW * 4 + 2 * bt * 4; }
+
+__host__ __device__ constexpr int smem_total(int mode, int bt, int stages) {
+  return 1024 + stages * stage_bytes(mode, bt) + kCSlots * cslot_bytes(bt) +
+         (3 * kMaxStages + 2 * kCSlots + 2 * kAccBufs) * 8 + 16;
+}
+
+// d.{x,y} = a.{x,y} + b.{x,y} and d = a * b + c on float pairs (one packed
+// f32x2 instruction each).
+__device__ __forceinline__ void add2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+template <int MODE, int BT, bool ACTG, bool DEBUG>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_linear_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_hi,
                      const __grid_constant__ CUtensorMap tm_lo, const Params p) {
   constexpr int OFF = CodeOffset<MODE>::value;
-  constexpr int COLS = BT / 2;            // columns per epilogue warp
+  constexpr int COLS = BT / 2;               // columns per epilogue warp
   constexpr int CH = COLS < 32 ? COLS : 32;  // columns per TMEM load
   constexpr uint32_t IDESC = umma_idesc_u8s8(BW, BT);
   constexpr int TCOLS = tmem_cols(BT);
+  constexpr int STAGE = stage_bytes(MODE, BT);
+  constexpr int CSLOT = cslot_bytes(BT);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   const int S = p.stages, G = p.G;
-  const Layout L = smem_layout(MODE, BT, S, G, p.sc_pitch);
-  uint8_t *sA = smem + L.a;
-  uint8_t *sB = smem + L.b;
-  uint8_t *sH = smem + L.h;
-  uint8_t *sL = smem + L.l;
-  __half *sSc = reinterpret_cast<__half *>(smem + L.sc);
-  int32_t *sCv = reinterpret_cast<int32_t *>(smem + L.cv);
-  float *sXv = reinterpret_cast<float *>(smem + L.xv);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
-  uint64_t *fullIn = bars;                    // TMA landed (q, hi, lo)
-  uint64_t *emptyIn = bars + kMaxStages;      // MMA done with the stage
-  uint64_t *fullA = bars + 2 * kMaxStages;    // transformed operand written
-  uint64_t *fullC = bars + 3 * kMaxStages;    // column constants written
-  uint64_t *emptyC = bars + 4 * kMaxStages;   // epilogue done with the constants
-  uint64_t *accFull = bars + 5 * kMaxStages;  // [2] accumulator ready
-  uint64_t *accEmpty = accFull + 2;           // [2] accumulator drained
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(accEmpty + 2);
+  // stage s: [A 16 KB][B bt x 128][hi 8 KB][lo 8 KB]
+  auto sA = [&](int s) { return smem + s * STAGE; };
+  auto sB = [&](int s) { return smem + s * STAGE + BW * 128; };
+  auto sH = [&](int s) { return smem + s * STAGE + BW * 128 + BT * 128; };
+  auto sL = [&](int s) { return smem + s * STAGE + BW * 128 + BT * 128 + BW * 64; };
+  // constant slot c: [row scales][column constants][act. scales]
+  uint8_t *cbase = smem + S * STAGE;
+  auto sSg = [&](int c) { return reinterpret_cast<float *>(cbase + c * CSLOT); };
+  auto sCv = [&](int c) { return reinterpret_cast<int32_t *>(sSg(c) + BW); };
+  auto sXv = [&](int c) { return reinterpret_cast<float *>(sCv(c) + BT); };
+  uint64_t *bars = reinterpret_cast<uint64_t *>(cbase + kCSlots * CSLOT);
+  uint64_t *fullB = bars;                      // activation and plane tiles landed
+  uint64_t *fullA = bars + kMaxStages;         // byte operand written
+  uint64_t *stageFree = bars + 2 * kMaxStages; // MMAs done with the stage
+  uint64_t *fullC = bars + 3 * kMaxStages;     // [kCSlots] per-group constants written
+  uint64_t *emptyC = fullC + kCSlots;          // [kCSlots] epilogue done with them
+  uint64_t *accFull = emptyC + kCSlots;        // [kAccBufs] accumulator ready
+  uint64_t *accEmpty = accFull + kAccBufs;     // [kAccBufs] accumulator drained
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(accEmpty + kAccBufs);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BW, m0 = blockIdx.y * BT;
+  const int mt = p.mt;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&fullIn[s], 1);
-      mbar_init(&emptyIn[s], 1);
+      mbar_init(&fullB[s], 1);
       mbar_init(&fullA[s], kNumXf);
-      mbar_init(&fullC[s], 1);
-      mbar_init(&emptyC[s], kNumEpi);
+      mbar_init(&stageFree[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int c = 0; c < kCSlots; ++c) {
+      mbar_init(&fullC[c], 1);
+      mbar_init(&emptyC[c], kNumEpi);
+    }
+    for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(&accFull[b], 1);
       mbar_init(&accEmpty[b], kNumEpi);
     }
@@ -145,175 +169,250 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tslot, TCOLS);
     tmem_relinquish();
   }
-  if (warp >= kWarpEpi0 && !DEBUG) {
-    // stage this tile's group scales, [row][pitch] fp16 (odd word pitch: the
-    // per-group column reads of 32 rows hit 32 different banks)
-    const int t = threadIdx.x - kWarpEpi0 * 32;
-    for (int i = t; i < BW * G; i += kNumEpi * 32) {
-      const int r = i / G, g = i - r * G;
-      const int n = n0 + r;
-      const uint16_t v = n < p.N ? __ldg(p.scale + (int64_t)n * G + g) : (uint16_t)0;
-      sSc[r * p.sc_pitch + g] = __ushort_as_half(v);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // the next kernel may start its prologue; the activations, their sums and
+  // scales come from the preceding one (waited for below, before each read)
+  griddep_launch_dependents();
 
-  if (warp == kWarpTma) {
-    // ------------------------------------------------------ TMA producer
+  if (warp < kWarpXf0 + kNumXf) {
+    // ---------------------------------------------- plane -> operand bytes
+    // thread t: rows pass * 32 + t / 4 (pass 0..3), 16-byte plane chunk
+    // t % 4 of the group (32 columns) -> 32 operand bytes of that row
+    const int t = threadIdx.x - kWarpXf0 * 32;  // 0..127
+    const int qd = t & 3;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+      for (int g = 0; g < G; ++g, ++it) {
+        const int s = it % S;
+        ok = mbar_wait_warp(&fullB[s], (it / S) & 1);
+        if (!ok) break;
+        const uint8_t *hs = sH(s);
+        const uint8_t *ls = sL(s);
+        uint8_t *as = sA(s);
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) {
+          const int r = pass * 32 + (t >> 2);
+          const uint4 h = *reinterpret_cast<const uint4 *>(hs + r * 64 + qd * 16);
+          uint4 l = make_uint4(0, 0, 0, 0);
+          if (MODE) l = *reinterpret_cast<const uint4 *>(ls + r * 64 + qd * 16);
+          const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+          const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
+          uint32_t out[8];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint32_t ev, od;  // bytes of columns 8w + {0,2,4,6} and 8w + {1,3,5,7}
+            if (MODE == 0) {
+              ev = hw[w] & 0x0F0F0F0Fu;
+              od = (hw[w] >> 4) & 0x0F0F0F0Fu;
+            } else {
+              ev = ((hw[w] << 4) & 0xF0F0F0F0u) | (lw[w] & 0x0F0F0F0Fu);
+              od = (hw[w] & 0xF0F0F0F0u) | ((lw[w] >> 4) & 0x0F0F0F0Fu);
+            }
+            out[2 * w] = prmt(ev, od, 0x5140);      // columns 8w + 0..3
+            out[2 * w + 1] = prmt(ev, od, 0x7362);  // columns 8w + 4..7
+          }
+          // 16-byte chunks 2qd and 2qd+1 of the 128-byte row, 128-byte swizzle
+          const int c0 = 2 * qd, c1 = 2 * qd + 1;
+          *reinterpret_cast<uint4 *>(as + r * 128 + ((c0 ^ (r & 7)) << 4)) =
+              make_uint4(out[0], out[1], out[2], out[3]);
+          *reinterpret_cast<uint4 *>(as + r * 128 + ((c1 ^ (r & 7)) << 4)) =
+              make_uint4(out[4], out[5], out[6], out[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&fullA[s]);
+      }
+    }
+  } else if (warp == kWarpTma) {
+    // --------------------------------------------------------- TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_hi);
       if (MODE) prefetch_tmap(&tm_lo);
-      const uint32_t bytes = BT * 128 + BW * 64 * (MODE ? 2 : 1);
-      int issued = 0;
-      for (int g = 0; g < G; ++g) {
-        const int s = g % S;
-        if (!mbar_wait(&emptyIn[s], ((g / S) & 1) ^ 1)) break;
-        mbar_arrive_expect_tx(&fullIn[s], bytes);
-        tma_load_2d(sB + s * BT * 128, &tm_q, &fullIn[s], g * 128, m0);
-        tma_load_2d(sH + s * BW * 64, &tm_hi, &fullIn[s], g * 64, n0);
-        if (MODE) tma_load_2d(sL + s * BW * 64, &tm_lo, &fullIn[s], g * 64, n0);
-        ++issued;
+      griddep_wait();
+      int it = 0;
+      bool ok = true;
+      constexpr uint32_t bytes = BT * 128 + BW * 64 * (MODE ? 2 : 1);
+      for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+        const int n0 = (tile / mt) * BW, m0 = (tile % mt) * BT;
+        for (int g = 0; g < G; ++g, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&stageFree[s], ((it / S) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&fullB[s], bytes);
+          tma_load_2d(sB(s), &tm_q, &fullB[s], g * 128, m0);
+          tma_load_2d(sH(s), &tm_hi, &fullB[s], g * 64, n0);
+          if (MODE) tma_load_2d(sL(s), &tm_lo, &fullB[s], g * 64, n0);
+        }
       }
-      if (issued < G) {  // gave up: let the copies already issued land
-        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
-          mbar_wait(&fullIn[i % S], (i / S) & 1);
-      }
+      if (!ok)  // gave up: let the copies already issued land
+        for (int i = (it > S ? it - S : 0); i < it; ++i) mbar_wait(&fullB[i % S], (i / S) & 1);
     }
   } else if (warp == kWarpMma) {
-    // ------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      int it = 0;
       bool ok = true;
-      for (int g = 0; g < G && ok; ++g) {
-        const int s = g % S, b = g & 1;
-        ok = mbar_wait(&fullA[s], (g / S) & 1) && mbar_wait(&accEmpty[b], ((g >> 1) & 1) ^ 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t ad = umma_desc_sw128(sA + s * BW * 128);
-        const uint64_t bd = umma_desc_sw128(sB + s * BT * 128);
+      for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+        for (int g = 0; g < G; ++g, ++it) {
+          const int s = it % S, b = it % kAccBufs;
+          ok = mbar_wait(&fullB[s], (it / S) & 1) && mbar_wait(&fullA[s], (it / S) & 1) &&
+               mbar_wait(&accEmpty[b], ((it / kAccBufs) & 1) ^ 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t ad = umma_desc_sw128(sA(s));
+          const uint64_t bd = umma_desc_sw128(sB(s));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // 4 x K=32 bytes inside the 128-byte row
-          umma_i8(tmem + b * BT, ad + 2 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
-        umma_commit(&emptyIn[s]);
-        umma_commit(&accFull[b]);
+          for (int kk = 0; kk < 4; ++kk)  // 4 x K=32 bytes inside the 128-byte row
+            umma_i8(tmem + b * BT, ad + 2 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
+          umma_commit(&stageFree[s]);
+          umma_commit(&accFull[b]);
+        }
       }
       // the last accumulator must be complete before TMEM is released
-      if (ok && G > 0) mbar_wait(&accFull[(G - 1) & 1], ((G - 1) >> 1) & 1);
+      if (ok && it > 0) mbar_wait(&accFull[(it - 1) % kAccBufs], ((it - 1) / kAccBufs) & 1);
     }
   } else if (warp == kWarpPrep) {
-    // ------------------------------------- per-group column constants
-    for (int g = 0; g < G; ++g) {
-      const int s = g % S;
-      if (!mbar_wait_warp(&emptyC[s], ((g / S) & 1) ^ 1)) break;
-      for (int j = lane; j < BT; j += 32) {
-        const int m = m0 + j;
-        const int r = m < p.M ? __ldg(p.xsum + (int64_t)m * G + g) : 0;
-        sCv[s * BT + j] = kMagicI - OFF * r;
-        if (p.act_group) sXv[s * BT + j] = m < p.M ? __ldg(p.xscale + (int64_t)m * G + g) : 0.0f;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&fullC[s]);
-    }
-  } else if (warp < kWarpEpi0) {
-    // ------------------------------------------ plane -> operand bytes
-    const int t = threadIdx.x - kWarpXf0 * 32;  // 0..127
-    const int qd = t & 3;                         // 32-column quarter of the group
-    for (int g = 0; g < G; ++g) {
-      const int s = g % S;
-      if (!mbar_wait_warp(&fullIn[s], (g / S) & 1)) break;
-      const uint8_t *hs = sH + s * BW * 64;
-      const uint8_t *ls = sL + s * BW * 64;
-      uint8_t *as = sA + s * BW * 128;
+    // ----------------------------------------------- per-group constants
+    // Eight groups per round trip: lane i holds rows i + 32 r (r < 4) and
+    // tokens i + 32 u (u < BT / 32, at least one), all loads of a batch
+    // issued before the first use.
+    constexpr int TU = BT < 32 ? 1 : BT / 32;
+    griddep_wait();
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+      const int n0 = (tile / mt) * BW, m0 = (tile % mt) * BT;
+      for (int gb = 0; gb < G && ok; gb += kCBatch) {
+        uint16_t sv[4][kCBatch];
+        int rv[TU][kCBatch];
+        float xv[TU][kCBatch];
 #pragma unroll
-      for (int pass = 0; pass < 4; ++pass) {
-        const int r = pass * 32 + (t >> 2);
-        const uint4 h = *reinterpret_cast<const uint4 *>(hs + r * 64 + qd * 16);
-        uint4 l = make_uint4(0, 0, 0, 0);
-        if (MODE) l = *reinterpret_cast<const uint4 *>(ls + r * 64 + qd * 16);
-        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
-        const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
-        uint32_t out[8];
+        for (int r = 0; r < 4; ++r) {
+          const int n = n0 + lane + 32 * r;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          uint32_t ev, od;  // bytes of columns 8w + {0,2,4,6} and 8w + {1,3,5,7}
-          if (MODE == 0) {
-            ev = hw[w] & 0x0F0F0F0Fu;
-            od = (hw[w] >> 4) & 0x0F0F0F0Fu;
-          } else {
-            ev = ((hw[w] << 4) & 0xF0F0F0F0u) | (lw[w] & 0x0F0F0F0Fu);
-            od = (hw[w] & 0xF0F0F0F0u) | ((lw[w] >> 4) & 0x0F0F0F0Fu);
-          }
-          out[2 * w] = prmt(ev, od, 0x5140);      // columns 8w + 0..3
-          out[2 * w + 1] = prmt(ev, od, 0x7362);  // columns 8w + 4..7
+          for (int k = 0; k < kCBatch; ++k)
+            sv[r][k] = (!DEBUG && n < p.N && gb + k < G) ? __ldg(p.scale + (int64_t)n * G + gb + k)
+                                                          : (uint16_t)0;
         }
-        // 16-byte chunks 2qd and 2qd+1 of the 128-byte row, 128-byte swizzle
-        const int c0 = 2 * qd, c1 = 2 * qd + 1;
-        *reinterpret_cast<uint4 *>(as + r * 128 + ((c0 ^ (r & 7)) << 4)) =
-            make_uint4(out[0], out[1], out[2], out[3]);
-        *reinterpret_cast<uint4 *>(as + r * 128 + ((c1 ^ (r & 7)) << 4)) =
-            make_uint4(out[4], out[5], out[6], out[7]);
+#pragma unroll
+        for (int u = 0; u < TU; ++u) {
+          const int j = lane + 32 * u, m = m0 + j;
+          const bool in = j < BT && m < p.M;
+#pragma unroll
+          for (int k = 0; k < kCBatch; ++k) {
+            rv[u][k] = (in && gb + k < G) ? __ldg(p.xsum + (int64_t)m * G + gb + k) : 0;
+            xv[u][k] = (ACTG && in && gb + k < G) ? __ldg(p.xscale + (int64_t)m * G + gb + k)
+                                                  : 0.0f;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kCBatch; ++k) {
+          if (gb + k >= G) break;
+          const int c = it % kCSlots;
+          ok = mbar_wait_warp(&emptyC[c], ((it / kCSlots) & 1) ^ 1);
+          if (!ok) break;
+          float *sg = sSg(c);
+          int32_t *cv = sCv(c);
+          float *xs = sXv(c);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) sg[lane + 32 * r] = __half2float(__ushort_as_half(sv[r][k]));
+#pragma unroll
+          for (int u = 0; u < TU; ++u) {
+            const int j = lane + 32 * u;
+            if (j < BT) {
+              cv[j] = kMagicI - OFF * rv[u][k];
+              if (ACTG) xs[j] = xv[u][k];
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&fullC[c]);
+          ++it;
+        }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&fullA[s]);
     }
   } else {
-    // --------------------------------------------------------- epilogue
+    // -------------------------------------------------------------- epilogue
     const int e = warp - kWarpEpi0;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int half = e >> 2;
     const int row = quarter * 32 + lane;
-    const int n = n0 + row;
     const int col0 = half * COLS;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    float acc[COLS];
+    griddep_wait();  // y may still be read by the preceding kernel
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+      const int n = (tile / mt) * BW + row, m0 = (tile % mt) * BT;
+      float acc[COLS];
 #pragma unroll
-    for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
-    for (int g = 0; g < G; ++g) {
-      const int s = g % S, b = g & 1;
-      if (!mbar_wait_warp(&fullC[s], (g / S) & 1)) break;
-      if (!mbar_wait_warp(&accFull[b], (g >> 1) & 1)) break;
-      tc_fence_after();
-      const float sg = DEBUG ? 0.0f : __half2float(sSc[row * p.sc_pitch + g]);
-      const int32_t *cv = sCv + s * BT + col0;
-      const float *xv = sXv + s * BT + col0;
+      for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
+      for (int g = 0; g < G; ++g, ++it) {
+        const int cs = it % kCSlots, b = it % kAccBufs;
+        ok = mbar_wait_warp(&fullC[cs], (it / kCSlots) & 1) &&
+             mbar_wait_warp(&accFull[b], (it / kAccBufs) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const float sg = sSg(cs)[row];
+        const int32_t *cv = sCv(cs) + col0;
+        const float *xv = sXv(cs) + col0;
 #pragma unroll
-      for (int c = 0; c < COLS; c += CH) {
-        uint32_t d[CH];
-        tmem_ld<CH>(tmem + lane_addr + b * BT + col0 + c, d);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < CH; ++j) {
-          const int bits = (int)d[j] + cv[c + j];  // 1.5 * 2^23 + exact group sum
+        for (int c = 0; c < COLS; c += CH) {
+          uint32_t d[CH];
+          tmem_ld<CH>(tmem + lane_addr + b * BT + col0 + c, d);
+          tmem_ld_wait();
           if (DEBUG) {
-            const int m = m0 + col0 + c + j;
-            if (m < p.M && n < p.N) p.S[((int64_t)m * p.N + n) * G + g] = bits - kMagicI;
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+              const int m = m0 + col0 + c + j;
+              if (m < p.M && n < p.N)
+                p.S[((int64_t)m * p.N + n) * G + g] = (int)d[j] + cv[c + j] - kMagicI;
+            }
           } else {
-            const float f = __int_as_float(bits) - kMagicF;
-            acc[c + j] = p.act_group ? fmaf(f, sg * xv[c + j], acc[c + j])
-                                     : fmaf(f, sg, acc[c + j]);
+#pragma unroll
+            for (int j = 0; j < CH; j += 4) {
+              const int4 c4 = *reinterpret_cast<const int4 *>(cv + c + j);
+              // 1.5 * 2^23 + exact group sum, as a float, minus the magic
+              float f0 = __int_as_float((int)d[j] + c4.x), f1 = __int_as_float((int)d[j + 1] + c4.y);
+              float f2 = __int_as_float((int)d[j + 2] + c4.z), f3 = __int_as_float((int)d[j + 3] + c4.w);
+              add2(f0, f1, f0, f1, -kMagicF, -kMagicF);
+              add2(f2, f3, f2, f3, -kMagicF, -kMagicF);
+              float s0 = sg, s1 = sg, s2 = sg, s3 = sg;
+              if (ACTG) {
+                const float4 x4 = *reinterpret_cast<const float4 *>(xv + c + j);
+                s0 *= x4.x;
+                s1 *= x4.y;
+                s2 *= x4.z;
+                s3 *= x4.w;
+              }
+              fma2(acc[c + j], acc[c + j + 1], f0, f1, s0, s1, acc[c + j], acc[c + j + 1]);
+              fma2(acc[c + j + 2], acc[c + j + 3], f2, f3, s2, s3, acc[c + j + 2], acc[c + j + 3]);
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&accEmpty[b]);
+          mbar_arrive(&emptyC[cs]);
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&accEmpty[b]);
-        mbar_arrive(&emptyC[s]);
-      }
-    }
-    if (!DEBUG && n < p.N) {
-      const float bias = p.bias ? __half2float(__ushort_as_half(__ldg(p.bias + n))) : 0.0f;
+      if (!DEBUG && ok && n < p.N) {
+        const float bias = p.bias ? __half2float(__ushort_as_half(__ldg(p.bias + n))) : 0.0f;
 #pragma unroll
-      for (int j = 0; j < COLS; ++j) {
-        const int m = m0 + col0 + j;
-        if (m < p.M) {
-          float out = p.act_group ? acc[j] : acc[j] * __ldg(p.xscale + m);
-          if (MODE) out *= 0.0625f;
-          p.y[(int64_t)m * p.N + n] = out + bias;
+        for (int j = 0; j < COLS; ++j) {
+          const int m = m0 + col0 + j;
+          if (m < p.M) {
+            float out = ACTG ? acc[j] : acc[j] * __ldg(p.xscale + m);
+            if (MODE) out *= 0.0625f;
+            p.y[(int64_t)m * p.N + n] = out + bias;
+          }
         }
       }
     }
@@ -364,32 +463,30 @@ int pick_bt(int64_t M) {
   return 128;
 }
 
-int sc_pitch(int G) {
-  int words = (G + 1) / 2;
-  words |= 1;  // odd number of 32-bit words per row
-  return 2 * words;
-}
-
-int pick_stages(int mode, int bt, int G, int max_smem) {
+int pick_stages(int mode, int bt, int max_smem) {
   for (int s = kMaxStages; s >= 2; --s)
-    if (smem_layout(mode, bt, s, G, sc_pitch(G)).total <= max_smem) return s;
+    if (smem_total(mode, bt, s) <= max_smem) return s;
   return 0;
 }
 
 constexpr int kMaxSmem = 227 * 1024;
 
-template <int MODE, int BT, bool DEBUG>
+int num_sms() {
+  static int sms[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  return sms[dev] > 0 ? sms[dev] : 148;
+}
+
+template <int MODE, int BT, bool ACTG, bool DEBUG>
 cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   const int G = (int)(a.K / kGroup);
-  const int stages = pick_stages(MODE, BT, G, kMaxSmem);
+  const int stages = pick_stages(MODE, BT, kMaxSmem);
   if (stages == 0) return cudaErrorInvalidValue;
-  const int pitch = sc_pitch(G);
-  const Layout L = smem_layout(MODE, BT, stages, G, pitch);
   CUtensorMap mq, mh, ml;
-  if (!make_map(&mq, a.xq, (uint64_t)a.M, (uint64_t)a.K, BT, 128,
-                CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mh, a.hi, (uint64_t)a.N, (uint64_t)(a.K / 2), BW, 64,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_map(&mq, a.xq, (uint64_t)a.M, (uint64_t)a.K, BT, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&mh, a.hi, (uint64_t)a.N, (uint64_t)(a.K / 2), BW, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   if (MODE) {
     if (!make_map(&ml, a.lo, (uint64_t)a.N, (uint64_t)(a.K / 2), BW, 64,
@@ -407,25 +504,37 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   p.S = a.S;
   p.M = (int)a.M;
   p.N = (int)a.N;
+  p.K = (int)a.K;
   p.G = G;
-  p.act_group = a.act_group;
+  p.mt = (int)((a.M + BT - 1) / BT);
+  const int64_t tiles = ((a.N + BW - 1) / BW) * (int64_t)p.mt;
+  if (tiles > (1 << 30)) return cudaErrorInvalidValue;
+  p.tiles = (int)tiles;
   p.stages = stages;
-  p.sc_pitch = pitch;
-  auto kern = tc_linear_kernel<MODE, BT, DEBUG>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  const int grid = p.tiles < num_sms() ? p.tiles : num_sms();
+  const int smem = smem_total(MODE, BT, stages);
+  auto kern = tc_linear_kernel<MODE, BT, ACTG, DEBUG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((a.N + BW - 1) / BW), (unsigned)((a.M + BT - 1) / BT));
-  kern<<<grid, kThreads, L.total, st>>>(mq, mh, ml, p);
+  e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, a.overlap, mq, mh,
+                 ml, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <int MODE, int BT, bool DEBUG>
+cudaError_t launch_g(const LinearArgs &a, cudaStream_t st) {
+  if (a.act_group != 0 && !DEBUG) return launch_t<MODE, BT, true, DEBUG>(a, st);
+  return launch_t<MODE, BT, false, DEBUG>(a, st);
 }
 
 template <int MODE, bool DEBUG>
 cudaError_t launch_mode(const LinearArgs &a, cudaStream_t st) {
   switch (pick_bt(a.M)) {
-    case 16: return launch_t<MODE, 16, DEBUG>(a, st);
-    case 32: return launch_t<MODE, 32, DEBUG>(a, st);
-    case 64: return launch_t<MODE, 64, DEBUG>(a, st);
-    default: return launch_t<MODE, 128, DEBUG>(a, st);
+    case 16: return launch_g<MODE, 16, DEBUG>(a, st);
+    case 32: return launch_g<MODE, 32, DEBUG>(a, st);
+    case 64: return launch_g<MODE, 64, DEBUG>(a, st);
+    default: return launch_g<MODE, 128, DEBUG>(a, st);
   }
 }
 
@@ -440,8 +549,8 @@ cudaError_t read_wait_timeout(int *flag, bool reset) {
 
 bool tc_supported(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || M > (int64_t)1 << 30 || N > (int64_t)1 << 30) return false;
-  const int G = (int)(K / kGroup);
-  return tc::pick_stages(1, tc::pick_bt(M), G, tc::kMaxSmem) >= 2;
+  if (K < kGroup || K % kGroup != 0 || K > ((int64_t)1 << 30)) return false;
+  return tc::pick_stages(1, tc::pick_bt(M), tc::kMaxSmem) >= 2;
 }
 
 cudaError_t launch_tc(const LinearArgs &a, cudaStream_t st) {
