@@ -62,6 +62,15 @@ def quant_bytes(M, K, act_group):
     return 2 * M * K + M * K + 4 * (M if act_group == 0 else M * G) + 4 * M * G
 
 
+def fused_bytes(mode, M, N, K, act_group):
+    """Algorithmic bytes of one quantise + linear call (bitnest_quantize_linear):
+    planes, fp16 group scales, fp16 activations read; int8 codes, their scales
+    and group sums, and the fp32 output written."""
+    G = K // 128
+    planes = (1 if mode == 0 else 2) * N * K // 2
+    return planes + 2 * N * G + quant_bytes(M, K, act_group) + 4 * M * N
+
+
 class ClockSampler:
     """NVML samples of SM clock and throttle reasons while the timed region runs."""
 
@@ -166,7 +175,7 @@ def decode_step_bytes():
     for _, members in LAYER_GROUPS:
         N, K, g = group_shape(members)
         for mode, M in DECODE_M.items():
-            tot += linear_bytes(mode, M, N, K) + quant_bytes(M, K, g)
+            tot += fused_bytes(mode, M, N, K, g)
     return tot
 
 
@@ -235,7 +244,7 @@ class DecodeWorkload:
         return decode_step_bytes()
 
     def launches_per_step(self):
-        return 2 * 2 * len(LAYER_GROUPS)
+        return 2 * len(LAYER_GROUPS)  # one quantise + linear kernel per layer group and pass
 
     def io_bytes(self):
         h2d = sum(t.numel() * t.element_size() for t in self.x_host.values())
@@ -245,11 +254,11 @@ class DecodeWorkload:
     def _path(self):
         return self.bn.PATH_AUTO | (self.bn.PATH_OVERLAP if self.overlap else 0)
 
-    def run_step(self, copy, events=None, e2e=False, qevents=None):
+    def run_step(self, copy, events=None, e2e=False):
         """Enqueue one step on the current stream: the draft pass then the
-        verify pass, each quantise + linear for the four layer groups.
-        `events` / `qevents`: per (group, mode) (start, end) CUDA events around
-        the linear / the quantiser."""
+        verify pass, one quantise + linear call (bitnest_quantize_linear) per
+        layer group.  `events`: per (group, mode) (start, end) CUDA events
+        around the call."""
         bn = self.bn
         w = self.copies[copy]
         for mode in (0, 1):
@@ -259,30 +268,25 @@ class DecodeWorkload:
                 x = self.x[gname, mode]
                 if e2e:
                     x.copy_(self.x_host[gname, mode], non_blocking=True)
-                if qevents is not None:
-                    qevents[gname, mode][0].record()
-                bn.quantize_act(x, g, out=(b["xq"], b["xs"], b["xsum"]))
-                if qevents is not None:
-                    qevents[gname, mode][1].record()
                 hi, lo, s = w[gname]
                 if events is not None:
                     events[gname, mode][0].record()
-                bn.linear(mode, hi, lo, s, b["xq"], b["xs"], b["xsum"], g, out=b["y"],
-                          path=self._path())
+                bn.quantize_linear(mode, hi, lo, s, x, g, out=b["y"],
+                                   act_out=(b["xq"], b["xs"], b["xsum"]), path=self._path())
                 if events is not None:
                     events[gname, mode][1].record()
                 if e2e:
                     b["y_host"].copy_(b["y"], non_blocking=True)
 
     def run_projection(self, name, mode):
-        """One unfused projection: quantise its own input, then the linear."""
+        """One unfused projection: quantise its own input and apply the layer."""
         bn = self.bn
         _, _, g = synth.LLAMA3_8B_PROJECTIONS[name]
         b = self.pbufs[name, mode]
-        bn.quantize_act(b["x"], g, out=(b["xq"], b["xs"], b["xsum"]))
         hi, lo, s = self.single[name]
-        return lambda: bn.linear(mode, hi, lo, s, b["xq"], b["xs"], b["xsum"], g, out=b["y"],
-                                 path=self._path())
+        return lambda: bn.quantize_linear(mode, hi, lo, s, b["x"], g, out=b["y"],
+                                          act_out=(b["xq"], b["xs"], b["xsum"]),
+                                          path=self._path())
 
 
 class EagerStep:
@@ -440,9 +444,8 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
         return {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for k in wl.bufs}
 
-    events, qevents = ev_pairs(), ev_pairs()
+    events = ev_pairs()
     dur = {k: 0.0 for k in events}
-    qdur = {k: 0.0 for k in events}
     n_ev = max(8, min(args.steps, 200))
     for i in range(n_ev):
         torch.cuda._sleep(4_000_000)
@@ -450,34 +453,23 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
         torch.cuda.synchronize()
         for k, (a, b) in events.items():
             dur[k] += a.elapsed_time(b) / 1e3
-    # the quantisers on their own pass (no events between them and their linear)
-    for i in range(n_ev):
-        torch.cuda._sleep(4_000_000)
-        wl.run_step(i % N_COPIES, qevents=qevents)
-        torch.cuda.synchronize()
-        for k, (a, b) in qevents.items():
-            qdur[k] += a.elapsed_time(b) / 1e3
     per_group = {}
     for (gname, mode) in events:
-        N, K, _ = group_shape(dict(LAYER_GROUPS)[gname])
+        N, K, g = group_shape(dict(LAYER_GROUPS)[gname])
         d = dur[gname, mode] / n_ev
-        b = linear_bytes(mode, DECODE_M[mode], N, K)
-        _, _, g = group_shape(dict(LAYER_GROUPS)[gname])
-        dq = qdur[gname, mode] / n_ev
+        b = fused_bytes(mode, DECODE_M[mode], N, K, g)
         per_group[f"{gname}/{'draft' if mode == 0 else 'target'}"] = {
             "N": N, "K": K, "us": round(d * 1e6, 3), "GB/s": round(b / d / 1e9, 1),
-            "frac_hbm": round(b / d / 1e9 / hbm_peak, 3),
-            "quantise_us": round(dq * 1e6, 3),
-            "quantise_GB/s": round(quant_bytes(DECODE_M[mode], K, g) / dq / 1e9, 1)}
-    # the dominant launch: the fused gate|up verify (target, M = 4) linear
-    dom_N, dom_K, _ = group_shape(dict(LAYER_GROUPS)["gate_up"])
-    dom_bytes = linear_bytes(1, DECODE_M[1], dom_N, dom_K)
+            "frac_hbm": round(b / d / 1e9 / hbm_peak, 3)}
+    # the dominant launch: the fused gate|up verify (target, M = 4) layer
+    dom_N, dom_K, dom_g = group_shape(dict(LAYER_GROUPS)["gate_up"])
+    dom_bytes = fused_bytes(1, DECODE_M[1], dom_N, dom_K, dom_g)
     dom_time = dur["gate_up", 1] / n_ev
     achieved = dom_bytes / dom_time / 1e9
     # every projection on its own (unfused), same events
     per_proj = {}
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for name, (N, K, _) in wl.projs:
+    for name, (N, K, g) in wl.projs:
         for mode, M in DECODE_M.items():
             t = 0.0
             reps = 20
@@ -490,13 +482,14 @@ def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind
                 torch.cuda.synchronize()
                 t += ev0.elapsed_time(ev1) / 1e3
             t /= reps
-            b = linear_bytes(mode, M, N, K)
+            b = fused_bytes(mode, M, N, K, g)
             per_proj[f"{name}/{'draft' if mode == 0 else 'target'}"] = {
                 "us": round(t * 1e6, 3), "GB/s": round(b / t / 1e9, 1),
                 "frac_hbm": round(b / t / 1e9 / hbm_peak, 3)}
     roofline = {
         "bound": "hbm",
-        "kernel": f"gemv_tma_kernel<TARGET, M=4>, fused gate|up (N={dom_N}, K={dom_K})",
+        "kernel": f"gemv_tma_kernel<TARGET, M=4, fused quantiser>, fused gate|up weights "
+                  f"(N={dom_N}, K={dom_K})",
         "achieved": round(achieved, 1),
         "peak": hbm_peak,
         "unit": "GB/s",
@@ -572,8 +565,7 @@ def round_bytes():
     """Algorithmic bytes of one speculative decode round over the 32 layers."""
     per = {}
     for mode, M in DECODE_M.items():
-        per[mode] = sum(linear_bytes(mode, M, *group_shape(m)[:2]) + quant_bytes(M, *group_shape(m)[1:])
-                        for _, m in LAYER_GROUPS)
+        per[mode] = sum(fused_bytes(mode, M, *group_shape(m)) for _, m in LAYER_GROUPS)
     return ROUND_LAYERS * (ROUND_DRAFT_PASSES * per[0] + per[1])
 
 
@@ -609,9 +601,9 @@ def measure_round(wl, hbm_peak, reps=10):
                 for gname, members in LAYER_GROUPS:
                     _, _, g = group_shape(members)
                     b = wl.bufs[gname, mode]
-                    bn.quantize_act(wl.x[gname, mode], g, out=(b["xq"], b["xs"], b["xsum"]))
                     hi, lo, s = lw[gname]
-                    bn.linear(mode, hi, lo, s, b["xq"], b["xs"], b["xsum"], g, out=b["y"], path=path)
+                    bn.quantize_linear(mode, hi, lo, s, wl.x[gname, mode], g, out=b["y"],
+                                       act_out=(b["xq"], b["xs"], b["xsum"]), path=path)
 
     graph = capture(one_round)
     for _ in range(3):
@@ -622,10 +614,10 @@ def measure_round(wl, hbm_peak, reps=10):
     del layers
     torch.cuda.empty_cache()
     nb = round_bytes()
-    launches = (ROUND_DRAFT_PASSES + 1) * ROUND_LAYERS * len(LAYER_GROUPS) * 2
+    launches = (ROUND_DRAFT_PASSES + 1) * ROUND_LAYERS * len(LAYER_GROUPS)
     return {
         "workload": "speculative round: 32 layers x 7 projections, 3 draft passes (M=1) + "
-                    "1 verify pass (M=4), quantisers included, one CUDA graph",
+                    "1 verify pass (M=4), one quantise + linear kernel per layer group, one CUDA graph",
         "us_per_round": round(t * 1e6, 1),
         "GB_per_round": round(nb / 1e9, 3),
         "GB_per_token_full_acceptance": round(nb / 1e9 / (ROUND_DRAFT_PASSES + 1), 3),
@@ -743,7 +735,7 @@ def main():
         "config": {
             "workload": wl_name,
             "projections": {k: list(v[:2]) for k, v in synth.LLAMA3_8B_PROJECTIONS.items()},
-            "launches": "per pass: quantise + linear for q|k|v (fused, N=6144), o (per-group "
+            "launches": "per pass: one quantise + linear kernel for q|k|v (fused, N=6144), o (per-group "
                         "activation scales), gate|up (fused, N=28672), down",
             "passes": "draft W4A8 M=1 then verify W8A8 M=4 (gamma+1)",
             "group": 128,

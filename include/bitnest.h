@@ -151,6 +151,24 @@ int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const ui
                         int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
                         int path, void *stream);
 
+/*
+ * Activation quantiser and nested linear layer in one call: the same results
+ * as bitnest_quantize_act(x, M, K, act_group, xq, xscale, xsum) followed by
+ * bitnest_linear_path(mode, hi, lo, scale, xq, xscale, xsum, M, N, K, y,
+ * act_group, bias, path), bit for bit in xq / xscale / xsum and y.
+ *   x                 : fp16 [M, K] activations (finite values).
+ *   xq, xscale, xsum  : outputs as in bitnest_quantize_act (all required).
+ * The quantiser and the layer kernel run back to back on `stream`; with
+ * BITNEST_PATH_OVERLAP the layer kernel streams its weights while the
+ * quantiser runs.  Argument checks and
+ * error behaviour are those of bitnest_linear_path plus: x non-NULL and
+ * 16-byte aligned.
+ */
+int bitnest_quantize_linear(int mode, const uint8_t *hi, const uint8_t *lo,
+                            const uint16_t *scale, const uint16_t *x, int64_t M, int64_t N,
+                            int64_t K, float *y, int act_group, const uint16_t *bias,
+                            int8_t *xq, float *xscale, int32_t *xsum, int path, void *stream);
+
 /* The kernel family BITNEST_PATH_AUTO picks for this problem (host only,
  * launches nothing).  Returns BITNEST_PATH_GEMV or BITNEST_PATH_TC. */
 int bitnest_select_path(int mode, int64_t M, int64_t N, int64_t K);

@@ -93,6 +93,27 @@ def test_linear_argument_checks(L):
     assert L.bitnest_device_wait_timeout is not None
 
 
+def test_quantize_linear_argument_checks(L):
+    v = ctypes.c_void_p
+
+    def q(x=A, xq=A, xs=A, xsum=A, M=4, N=64, K=128, mode=1, g=0, path=0):
+        return L.bitnest_quantize_linear(mode, v(A), v(A), v(A), v(x) if x else None, M, N, K,
+                                         v(A), g, None, v(xq) if xq else None,
+                                         v(xs) if xs else None, v(xsum) if xsum else None,
+                                         path, None)
+
+    assert q(x=0) == 1
+    assert q(x=MIS) == 3
+    assert q(xq=0) == 1
+    assert q(xsum=MIS) == 3
+    assert q(K=200) == 2
+    assert q(g=7) == 1
+    assert q(path=5) == 1
+    assert q(M=9, path=1) == 2  # GEMV takes at most 8 tokens: nothing launched
+    assert q(M=0) == 0
+    assert q(N=0) == 0
+
+
 def test_quantize_pack_sum_argument_checks(L):
     v = ctypes.c_void_p
     assert L.bitnest_quantize_act(v(A), 4, 128, 3, v(A), v(A), None, None) == 1

@@ -209,3 +209,55 @@ def test_gemv_simple_kernel_for_odd_k(M, N, K, mode):
         torch.cuda.synchronize()
         assert np.array_equal(host(S), oracle.group_sums(mode, p.hi, p.lo, p.q, KK))
         assert oracle.max_normalised_error(p.y_gpu(mode, bn.PATH_GEMV), p.y_ref(mode)) <= TOL
+
+
+# ------------------------------------------- fused quantiser + linear layer
+@pytest.mark.parametrize("M,N,K", [(1, 37, 1024), (4, 300, 4096), (3, 129, 2048), (8, 64, 1024),
+                                   (4, 200, 14336), (2, 50, 1152), (12, 130, 1024)])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("act_group", [0, 128])
+def test_quantize_linear_matches_oracle(M, N, K, mode, act_group):
+    """One call: the codes, scales and group sums are the quantiser's, bit for
+    bit; y matches the oracle, on the GEMV and the tensor-core paths."""
+    p = Problem(M, N, K, seed=7 * M + N, act_group=act_group)
+    for path in (bn.PATH_AUTO, bn.PATH_AUTO | bn.PATH_OVERLAP):
+        y, (xq, xs, xsum) = bn.quantize_linear(mode, p.d_hi, p.d_lo, p.d_s, p.d_x, act_group,
+                                               path=path)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(xq), p.q)
+        assert np.array_equal(host(xs), p.xs)
+        assert np.array_equal(host(xsum), p.q.astype(np.int64).reshape(M, K // 128, 128).sum(2))
+        assert oracle.max_normalised_error(host(y), p.y_ref(mode)) <= TOL
+    assert bn.device_wait_timeout(reset=True) == 0
+
+
+def _near_tie_activations(M, K, seed):
+    """Rows whose values land near and exactly on half-integers of x / s:
+    the quantiser's rounding is decided by the correctly rounded quotient."""
+    rng = np.random.default_rng(seed)
+    x = np.zeros((M, K), np.float16)
+    for m in range(M):
+        amax = np.float32(rng.uniform(0.5, 40.0))
+        s = np.float32(amax) / np.float32(127.0)
+        k = rng.integers(-126, 126, size=K).astype(np.float32) + np.float32(0.5)
+        jitter = rng.choice(np.array([0.0, 1e-4, -1e-4, 3e-5, -3e-5, 1e-6], np.float32), size=K)
+        x[m] = (k * (1.0 + jitter) * s).astype(np.float16)
+        x[m, rng.integers(0, K)] = np.float16(amax)
+    return x
+
+
+@pytest.mark.parametrize("act_group", [0, 128])
+def test_quantiser_near_ties_bit_exact(act_group):
+    for M, K in ((1, 4096), (4, 14336), (3, 1152)):
+        x = _near_tie_activations(M, K, seed=M + K + act_group)
+        q, xs = oracle.quantize(x, act_group)
+        d_xq, d_xs, _ = bn.quantize_act(dev(x), act_group)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(d_xq), q)
+        assert np.array_equal(host(d_xs), xs)
+        if M <= 8:  # the one-call quantise + layer entry point
+            p = Problem(M, 40, K, seed=3)
+            _, (fq, fs, _) = bn.quantize_linear(0, p.d_hi, p.d_lo, p.d_s, dev(x), act_group)
+            torch.cuda.synchronize()
+            assert np.array_equal(host(fq), q)
+            assert np.array_equal(host(fs), xs)

@@ -59,9 +59,10 @@ def lib() -> ctypes.CDLL:
     L.bitnest_linear_path.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, I, P]
     L.bitnest_select_path.argtypes = [I, I64, I64, I64]
     L.bitnest_debug_group_sums.argtypes = [I, P, P, P, P, I64, I64, I64, P, I, P]
+    L.bitnest_quantize_linear.argtypes = [I, P, P, P, P, I64, I64, I64, P, I, P, P, P, P, I, P]
     for name in ("bitnest_pack_planes", "bitnest_quantize_act", "bitnest_act_group_sums",
                  "bitnest_linear", "bitnest_linear_path", "bitnest_select_path",
-                 "bitnest_debug_group_sums"):
+                 "bitnest_debug_group_sums", "bitnest_quantize_linear"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -151,6 +152,30 @@ def linear(mode: int, hi, lo, scale, xq, xscale, xsum, act_group: int = 0, bias=
                                      _ptr(xscale), _ptr(xsum), M, N, K, _ptr(y), int(act_group),
                                      _ptr(bias), int(path), _stream(xq)), "bitnest_linear")
     return y
+
+
+def quantize_linear(mode: int, hi, lo, scale, x, act_group: int = 0, bias=None, out=None,
+                    act_out=None, path: int = PATH_AUTO):
+    """Quantise fp16 x [M, K] and apply the nested linear layer in one call.
+
+    Returns (y fp32 [M, N], (xq, xscale, xsum)); the activation outputs are
+    the same as quantize_act's.  `act_out` may supply their buffers."""
+    import torch
+
+    M, K = x.shape
+    N = hi.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
+    if act_out is None:
+        act_out = (torch.empty((M, K), dtype=torch.int8, device=x.device),
+                   torch.empty((M,) if act_group == 0 else (M, K // GROUP), dtype=torch.float32,
+                               device=x.device),
+                   torch.empty((M, K // GROUP), dtype=torch.int32, device=x.device))
+    xq, xs, xsum = act_out
+    _check(lib().bitnest_quantize_linear(int(mode), _ptr(hi), _ptr(lo), _ptr(scale), _ptr(x), M, N,
+                                         K, _ptr(y), int(act_group), _ptr(bias), _ptr(xq),
+                                         _ptr(xs), _ptr(xsum), int(path), _stream(x)),
+           "bitnest_quantize_linear")
+    return y, (xq, xs, xsum)
 
 
 def debug_group_sums(mode: int, hi, lo, xq, xsum, path: int = PATH_AUTO, out=None):

@@ -149,6 +149,31 @@ int bitnest_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_
                              bias, BITNEST_PATH_AUTO, stream);
 }
 
+int bitnest_quantize_linear(int mode, const uint8_t *hi, const uint8_t *lo,
+                            const uint16_t *scale, const uint16_t *x, int64_t M, int64_t N,
+                            int64_t K, float *y, int act_group, const uint16_t *bias,
+                            int8_t *xq, float *xscale, int32_t *xsum, int path, void *stream) {
+  const bool overlap = (path & BITNEST_PATH_OVERLAP) != 0;
+  path &= ~BITNEST_PATH_OVERLAP;
+  if (path < BITNEST_PATH_AUTO || path > BITNEST_PATH_TC) return BITNEST_ERR_INVALID_ARG;
+  int s = check_linear(mode, hi, lo, scale, xq, xscale, xsum, M, N, K, y, act_group, bias);
+  if (s != BITNEST_OK) return s;
+  if (M == 0 || N == 0) return BITNEST_OK;
+  if (!x) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(x)) return BITNEST_ERR_MISALIGNED;
+  cudaStream_t st = (cudaStream_t)stream;
+  LinearArgs a{mode, hi, mode == BITNEST_TARGET ? lo : nullptr, scale, xq, xscale, xsum,
+               bias, y, nullptr, M, N, K, act_group, overlap};
+  if (path == BITNEST_PATH_AUTO) path = pick_path(mode, M, N, K);
+  // the layer's shape is checked before anything is launched
+  if (path == BITNEST_PATH_GEMV && !gemv_tma_supported(M, N, K) && !gemv_fits(M, K))
+    return BITNEST_ERR_UNSUPPORTED_SHAPE;
+  if (path == BITNEST_PATH_TC && !tc_supported(M, N, K)) return BITNEST_ERR_UNSUPPORTED_SHAPE;
+  s = cuda_status(launch_quantize(x, M, K, act_group, xq, xscale, xsum, st));
+  if (s != BITNEST_OK) return s;
+  return run_linear(a, path, st);
+}
+
 int bitnest_debug_group_sums(int mode, const uint8_t *hi, const uint8_t *lo,
                              const int8_t *xq, const int32_t *xsum, int64_t M, int64_t N,
                              int64_t K, int32_t *S, int path, void *stream) {

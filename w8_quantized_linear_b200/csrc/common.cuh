@@ -83,6 +83,22 @@ inline cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cud
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// Symmetric int8 code of one activation (model table row "Activations"):
+// q = clamp(rne(x / s), -127, 127), with x / s the correctly rounded fp32
+// quotient and s = max|x| / 127 (so |x / s| <= 127.00001).  rs = RN(1 / s).
+// The product t = RN(x * rs) lies within 1.6e-5 of the exact quotient and
+// RN(x / s) within 3.9e-6 of it; so unless t is within 2^-15 of a
+// half-integer both round to the same integer, and only those rare values pay
+// for the correctly rounded division.
+__device__ __forceinline__ int quant_code(float x, float s, float rs) {
+  if (s == 0.0f) return 0;
+  const float t = __fmul_rn(x, rs);
+  const float frac = t - floorf(t);  // exact: |t| < 2^23
+  const int q = fabsf(frac - 0.5f) < 3.0517578125e-05f ? __float2int_rn(__fdiv_rn(x, s))
+                                                       : __float2int_rn(t);
+  return max(-127, min(127, q));
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

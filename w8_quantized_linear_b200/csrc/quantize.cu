@@ -32,23 +32,16 @@ cudaError_t launch_pack(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t
 }
 
 // ------------------------------------------------------------ quantiser
-// q = clamp(rne(x / s), -127, 127), s = max|x| / 127 (correctly rounded fp32
-// division); s == 0 gives q = 0.
-__device__ __forceinline__ int quant_one(float x, float s) {
-  if (s == 0.0f) return 0;
-  int q = __float2int_rn(__fdiv_rn(x, s));
-  return max(-127, min(127, q));
-}
-
-// Quantise 8 values (one 16-byte vector); returns the 8 codes packed and
-// adds their sum to *sum.
+// Quantise 8 values (one 16-byte vector) with scale s (s == 0 gives zeros);
+// returns the 8 codes packed and adds their sum to *sum.
 __device__ __forceinline__ uint2 quant8(const uint4 v, float s, int *sum) {
   const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+  const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     float2 f = __half22float2(h[i]);
-    int q0 = quant_one(f.x, s), q1 = quant_one(f.y, s);
+    int q0 = quant_code(f.x, s, rs), q1 = quant_code(f.y, s, rs);
     *sum += q0 + q1;
     uint32_t pair = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8);
     w[i >> 1] |= pair << (16 * (i & 1));
@@ -68,8 +61,10 @@ __device__ __forceinline__ float amax8(const uint4 v) {
 }
 
 // One block per token.  Vector v (8 columns) is handled by thread v % T; a
-// group (16 vectors) is 16 consecutive threads of one pass.
-template <int T>
+// group (16 vectors) is 16 consecutive threads of one pass.  With V > 0 every
+// thread holds its (at most V) vectors in registers: one read of x, one
+// block reduction of max|x|, then the codes.  V == 0 reads x twice (any K).
+template <int T, int V>
 __global__ void __launch_bounds__(T) quantize_token_kernel(const uint16_t *__restrict__ x,
                                                            int64_t K, int8_t *__restrict__ xq,
                                                            float *__restrict__ xs,
@@ -81,8 +76,20 @@ __global__ void __launch_bounds__(T) quantize_token_kernel(const uint16_t *__res
   const int64_t m = blockIdx.x;
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + m * K);
   const int nvec = (int)(K / 8);
+  constexpr int R = V > 0 ? V : 1;
+  uint4 v[R];
   float amax = 0.0f;
-  for (int v = threadIdx.x; v < nvec; v += T) amax = fmaxf(amax, amax8(__ldg(xr + v)));
+  if (V > 0) {
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const int i = threadIdx.x + j * T;
+      v[j] = i < nvec ? __ldg(xr + i) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < R; ++j) amax = fmaxf(amax, amax8(v[j]));
+  } else {
+    for (int i = threadIdx.x; i < nvec; i += T) amax = fmaxf(amax, amax8(__ldg(xr + i)));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   __shared__ float red[T / 32];
@@ -95,14 +102,23 @@ __global__ void __launch_bounds__(T) quantize_token_kernel(const uint16_t *__res
   if (threadIdx.x == 0) xs[m] = s;
   uint2 *qr = reinterpret_cast<uint2 *>(xq + m * K);
   const int G = (int)(K / kGroup);
-  for (int v0 = 0; v0 < nvec; v0 += T) {
-    const int v = v0 + threadIdx.x;
+  // codes of vector i (held in `val`) and the sum of its group
+  auto emit = [&](int i, const uint4 &val) {
     int sum = 0;
-    if (v < nvec) qr[v] = quant8(__ldg(xr + v), s, &sum);
+    if (i < nvec) qr[i] = quant8(val, s, &sum);
     // 16 consecutive threads hold one group (T is a multiple of 16, nvec of 16)
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (xsum && v < nvec && (v & 15) == 0) xsum[m * G + v / 16] = sum;
+    if (xsum && i < nvec && (i & 15) == 0) xsum[m * G + i / 16] = sum;
+  };
+  if (V > 0) {
+#pragma unroll
+    for (int j = 0; j < R; ++j) emit(threadIdx.x + j * T, v[j]);
+  } else {
+    for (int i0 = 0; i0 < nvec; i0 += T) {
+      const int i = i0 + threadIdx.x;
+      emit(i, i < nvec ? __ldg(xr + i) : make_uint4(0, 0, 0, 0));
+    }
   }
 }
 
@@ -141,8 +157,14 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t M, int64_t K, int act_gro
   // programmatic dependent launch: the kernel waits for its predecessor first
   cudaError_t e;
   if (act_group == 0) {
-    e = launch_pdl(quantize_token_kernel<512>, dim3((unsigned)M), dim3(512), 0, st, true, x, K, xq,
-                   xs, xsum);
+    constexpr int T = 256;
+    const int64_t per = (K / 8 + T - 1) / T;  // vectors per thread
+    auto kern = per <= 1 ? quantize_token_kernel<T, 1>
+                : per <= 2 ? quantize_token_kernel<T, 2>
+                : per <= 4 ? quantize_token_kernel<T, 4>
+                : per <= 8 ? quantize_token_kernel<T, 8>
+                : per <= 16 ? quantize_token_kernel<T, 16> : quantize_token_kernel<T, 0>;
+    e = launch_pdl(kern, dim3((unsigned)M), dim3(T), 0, st, true, x, K, xq, xs, xsum);
   } else {
     const int64_t nvec = M * K / 8;
     const int threads = 256;
