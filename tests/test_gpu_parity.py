@@ -213,12 +213,14 @@ def test_gemv_simple_kernel_for_odd_k(M, N, K, mode):
 
 # ------------------------------------------- fused quantiser + linear layer
 @pytest.mark.parametrize("M,N,K", [(1, 37, 1024), (4, 300, 4096), (3, 129, 2048), (8, 64, 1024),
-                                   (4, 200, 14336), (2, 50, 1152), (12, 130, 1024)])
+                                   (4, 200, 14336), (2, 50, 1152), (12, 130, 1024),
+                                   (4, 2500, 2048), (1, 2500, 3072), (7, 2400, 1024)])
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("act_group", [0, 128])
 def test_quantize_linear_matches_oracle(M, N, K, mode, act_group):
     """One call: the codes, scales and group sums are the quantiser's, bit for
-    bit; y matches the oracle, on the GEMV and the tensor-core paths."""
+    bit; y matches the oracle, on the GEMV and the tensor-core paths (N > 2368
+    gives the decode GEMV's CTAs more than one 16-row block each)."""
     p = Problem(M, N, K, seed=7 * M + N, act_group=act_group)
     for path in (bn.PATH_AUTO, bn.PATH_AUTO | bn.PATH_OVERLAP):
         y, (xq, xs, xsum) = bn.quantize_linear(mode, p.d_hi, p.d_lo, p.d_s, p.d_x, act_group,

@@ -4,6 +4,7 @@
 // o_proj).
 #include "common.cuh"
 #include "launch.h"
+#include "sm100.cuh"
 
 namespace bitnest {
 
@@ -32,34 +33,6 @@ cudaError_t launch_pack(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t
 }
 
 // ------------------------------------------------------------ quantiser
-// Quantise 8 values (one 16-byte vector) with scale s (s == 0 gives zeros);
-// returns the 8 codes packed and adds their sum to *sum.
-__device__ __forceinline__ uint2 quant8(const uint4 v, float s, int *sum) {
-  const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-  const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
-  uint32_t w[2] = {0u, 0u};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __half22float2(h[i]);
-    int q0 = quant_code(f.x, s, rs), q1 = quant_code(f.y, s, rs);
-    *sum += q0 + q1;
-    uint32_t pair = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8);
-    w[i >> 1] |= pair << (16 * (i & 1));
-  }
-  return make_uint2(w[0], w[1]);
-}
-
-__device__ __forceinline__ float amax8(const uint4 v) {
-  const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __half22float2(h[i]);
-    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-  }
-  return m;
-}
-
 // One block per token.  Vector v (8 columns) is handled by thread v % T; a
 // group (16 vectors) is 16 consecutive threads of one pass.  With V > 0 every
 // thread holds its (at most V) vectors in registers: one read of x, one
@@ -69,12 +42,19 @@ __global__ void __launch_bounds__(T) quantize_token_kernel(const uint16_t *__res
                                                            int64_t K, int8_t *__restrict__ xq,
                                                            float *__restrict__ xs,
                                                            int32_t *__restrict__ xsum) {
-  // x may come from the preceding kernel: wait for it, and only then let the
-  // next kernel (the layer, which may stream its weights early) start
-  griddep_wait();
-  griddep_launch_dependents();
   const int64_t m = blockIdx.x;
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + m * K);
+  // This block is resident while the preceding kernel runs: ask for the row
+  // in L2 now (a hint; the read below comes after the wait).  x may come
+  // from the preceding kernel: wait for it, and only then let the next kernel
+  // (the layer, which may stream its weights early) start.
+  if (threadIdx.x == 0) {
+    for (int64_t o = 0; o < K * 2; o += 65536)
+      prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(xr) + o,
+                       (uint32_t)(K * 2 - o < 65536 ? K * 2 - o : 65536));
+  }
+  griddep_wait();
+  griddep_launch_dependents();
   const int nvec = (int)(K / 8);
   constexpr int R = V > 0 ? V : 1;
   uint4 v[R];
@@ -99,13 +79,14 @@ __global__ void __launch_bounds__(T) quantize_token_kernel(const uint16_t *__res
 #pragma unroll
   for (int i = 1; i < T / 32; ++i) amax = fmaxf(amax, red[i]);
   const float s = __fdiv_rn(amax, 127.0f);
+  const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
   if (threadIdx.x == 0) xs[m] = s;
   uint2 *qr = reinterpret_cast<uint2 *>(xq + m * K);
   const int G = (int)(K / kGroup);
   // codes of vector i (held in `val`) and the sum of its group
   auto emit = [&](int i, const uint4 &val) {
     int sum = 0;
-    if (i < nvec) qr[i] = quant8(val, s, &sum);
+    if (i < nvec) qr[i] = quant8(val, s, rs, &sum);
     // 16 consecutive threads hold one group (T is a multiple of 16, nvec of 16)
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -128,10 +109,15 @@ __global__ void __launch_bounds__(256) quantize_group_kernel(const uint16_t *__r
                                                              int8_t *__restrict__ xq,
                                                              float *__restrict__ xs,
                                                              int32_t *__restrict__ xsum) {
-  griddep_wait();
-  griddep_launch_dependents();
   const int64_t nvec = M * K / 8;
   const int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // vectors in order
+  if (threadIdx.x == 0) {  // this block's slice into L2 before the wait (a hint)
+    const int64_t v0 = blockIdx.x * (int64_t)blockDim.x;
+    const int64_t n = (nvec - v0 < (int64_t)blockDim.x ? nvec - v0 : (int64_t)blockDim.x);
+    prefetch_l2_bulk(reinterpret_cast<const uint4 *>(x) + v0, (uint32_t)(n * 16));
+  }
+  griddep_wait();
+  griddep_launch_dependents();
   const bool ok = v < nvec;  // nvec is a multiple of 16: whole groups share `ok`
   uint4 val = ok ? __ldg(reinterpret_cast<const uint4 *>(x) + v) : make_uint4(0, 0, 0, 0);
   float amax = amax8(val);
@@ -139,7 +125,7 @@ __global__ void __launch_bounds__(256) quantize_group_kernel(const uint16_t *__r
   for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float s = __fdiv_rn(amax, 127.0f);
   int sum = 0;
-  uint2 q = quant8(val, s, &sum);
+  uint2 q = quant8(val, s, s == 0.0f ? 0.0f : __frcp_rn(s), &sum);
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (ok) {

@@ -77,6 +77,13 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, uint64_
       : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) into L2 (src 16-byte aligned, bytes a
+// multiple of 16).  A cache hint only: L2 is where global writes become
+// coherent, so a later read still sees data written after the prefetch.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
