@@ -48,7 +48,7 @@ constexpr int kCSlots = 16;    // per-group constant slots
 constexpr int kCBatch = 8;     // groups of constants per round trip
 constexpr int kWarpXf0 = 0, kNumXf = 4;
 constexpr int kWarpTma = 4, kWarpMma = 5, kWarpPrep = 6;
-constexpr int kWarpEpi0 = 7, kNumEpi = 8;
+constexpr int kWarpEpi0 = 7, kNumEpi = 8;  // two epilogue warps per TMEM lane quarter
 constexpr int kWarps = 15;
 constexpr int kThreads = kWarps * 32;
 // 1.5 * 2^23: adding an integer |s| < 2^22 to this bit pattern gives the
@@ -183,12 +183,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // t % 4 of the group (32 columns) -> 32 operand bytes of that row
     const int t = threadIdx.x - kWarpXf0 * 32;  // 0..127
     const int qd = t & 3;
-    int it = 0;
+    int s = 0;
+    uint32_t ph = 0;  // stage slot and the parity of its current fill
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-      for (int g = 0; g < G; ++g, ++it) {
-        const int s = it % S;
-        ok = mbar_wait_warp(&fullB[s], (it / S) & 1);
+      for (int g = 0; g < G; ++g) {
+        ok = mbar_wait_warp(&fullB[s], ph);
         if (!ok) break;
         const uint8_t *hs = sH(s);
         const uint8_t *ls = sL(s);
@@ -225,6 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&fullA[s]);
+        if (++s == S) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
     }
   } else if (warp == kWarpTma) {
@@ -234,14 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_hi);
       if (MODE) prefetch_tmap(&tm_lo);
       griddep_wait();
-      int it = 0;
+      int it = 0, s = 0;
+      uint32_t ph = 0;
       bool ok = true;
       constexpr uint32_t bytes = BT * 128 + BW * 64 * (MODE ? 2 : 1);
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
         const int n0 = (tile / mt) * BW, m0 = (tile % mt) * BT;
         for (int g = 0; g < G; ++g, ++it) {
-          const int s = it % S;
-          if (!mbar_wait(&stageFree[s], ((it / S) & 1) ^ 1)) {
+          if (!mbar_wait(&stageFree[s], ph ^ 1u)) {
             ok = false;
             break;
           }
@@ -249,6 +253,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sB(s), &tm_q, &fullB[s], g * 128, m0);
           tma_load_2d(sH(s), &tm_hi, &fullB[s], g * 64, n0);
           if (MODE) tma_load_2d(sL(s), &tm_lo, &fullB[s], g * 64, n0);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
       if (!ok)  // gave up: let the copies already issued land
@@ -257,26 +265,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int it = 0;
+      // every count, slot and descriptor is kept incrementally: this one
+      // thread shares its scheduler with busy warps, so each instruction it
+      // saves shortens the gap between two groups' MMAs
+      int s = 0, b = 0, it = 0;
+      uint32_t ph = 0, bph = 0;
+      const uint64_t ad0 = umma_desc_sw128(sA(0)), bd0 = umma_desc_sw128(sB(0));
+      constexpr uint64_t kStageDesc = STAGE >> 4;  // descriptor address unit: 16 bytes
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
         for (int g = 0; g < G; ++g, ++it) {
-          const int s = it % S, b = it % kAccBufs;
-          ok = mbar_wait(&fullB[s], (it / S) & 1) && mbar_wait(&fullA[s], (it / S) & 1) &&
-               mbar_wait(&accEmpty[b], ((it / kAccBufs) & 1) ^ 1);
+          ok = mbar_wait(&fullB[s], ph) && mbar_wait(&fullA[s], ph) &&
+               mbar_wait(&accEmpty[b], bph ^ 1u);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t ad = umma_desc_sw128(sA(s));
-          const uint64_t bd = umma_desc_sw128(sB(s));
+          const uint64_t ad = ad0 + (uint64_t)s * kStageDesc, bd = bd0 + (uint64_t)s * kStageDesc;
+          const uint32_t dt = tmem + (uint32_t)(b * BT);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // 4 x K=32 bytes inside the 128-byte row
-            umma_i8(tmem + b * BT, ad + 2 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
+            umma_i8(dt, ad + 2 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
           umma_commit(&stageFree[s]);
           umma_commit(&accFull[b]);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+          if (++b == kAccBufs) {
+            b = 0;
+            bph ^= 1u;
+          }
         }
       }
       // the last accumulator must be complete before TMEM is released
-      if (ok && it > 0) mbar_wait(&accFull[(it - 1) % kAccBufs], ((it - 1) / kAccBufs) & 1);
+      if (ok && it > 0) {
+        const int lb = b == 0 ? kAccBufs - 1 : b - 1;
+        mbar_wait(&accFull[lb], b == 0 ? bph ^ 1u : bph);
+      }
     }
   } else if (warp == kWarpPrep) {
     // ----------------------------------------------- per-group constants
