@@ -47,7 +47,8 @@ extern "C" {
 
 /* Kernel family for bitnest_linear_path. */
 #define BITNEST_PATH_AUTO 0 /* the library picks (see bitnest_select_path)          */
-#define BITNEST_PATH_GEMV 1 /* CUDA-core decode GEMV: dp4a, M <= BITNEST_GEMV_MAX_M  */
+#define BITNEST_PATH_GEMV 1 /* decode GEMV (planes streamed by TMA, integer
+                               mma.sync group sums), M <= BITNEST_GEMV_MAX_M */
 #define BITNEST_PATH_TC 2   /* tcgen05 kind::i8 tensor-core GEMM, any M              */
 
 #define BITNEST_GEMV_MAX_M 8 /* largest M the GEMV kernels are built for */
@@ -150,6 +151,36 @@ int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const ui
                         const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
                         int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
                         int path, void *stream);
+
+/*
+ * bitnest_linear_path with caller-provided scratch `ws` (device memory,
+ * 16-byte aligned, ws_bytes long) that the tensor-core path uses to split K
+ * when the layer has too few (row tile, token tile) pairs to fill the GPU
+ * (few output rows and tokens, long K: e.g. down_proj, N = 4096, K = 14336,
+ * at M <= 128).  The split ranges' fp32 partial sums go to ws; the last range
+ * to finish each sub-block adds them in a fixed order, so results do not
+ * depend on timing.  They agree with bitnest_linear_path's to within fp32
+ * summation rounding (the group sums themselves are the same exact int32).
+ *   ws, ws_bytes : at least bitnest_linear_ws_bytes(mode, M, N, K, path)
+ *                  bytes (BITNEST_ERR_INVALID_ARG if fewer).  When that is 0
+ *                  ws may be NULL and the call is bitnest_linear_path.
+ * The tail of ws holds arrival counters that must be zero before the first
+ * call (cudaMemset once); every call leaves them zero.  Calls sharing one ws
+ * must not run at the same time (calls in order on one stream are fine).
+ * With BITNEST_PATH_AUTO the choice may differ from bitnest_select_path's:
+ * where the TMA-ring GEMV does not apply and K would be split, the
+ * tensor-core path is taken (e.g. 5..8 tokens with K = 14336).
+ * Other arguments, checks and errors: as bitnest_linear_path.
+ */
+int bitnest_linear_ws(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                      const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
+                      int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
+                      int path, void *ws, int64_t ws_bytes, void *stream);
+
+/* Scratch bytes bitnest_linear_ws uses for this problem and path (0 when the
+ * path does not split K).  Host only; -BITNEST_ERR_INVALID_ARG for a bad
+ * mode or path, -BITNEST_ERR_UNSUPPORTED_SHAPE for a bad shape. */
+int64_t bitnest_linear_ws_bytes(int mode, int64_t M, int64_t N, int64_t K, int path);
 
 /*
  * Activation quantiser and nested linear layer in one call: the same results

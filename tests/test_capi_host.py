@@ -137,3 +137,31 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(bn, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         bn.lib()
+
+
+def test_linear_ws_argument_checks(L):
+    """Split-K scratch: its size query and the checks on it (no launch)."""
+    v = ctypes.c_void_p
+    need = L.bitnest_linear_ws_bytes(1, 16, 300, 1024, 2)
+    assert need > 0  # 3 weight tiles: the tensor-core path splits K
+    assert L.bitnest_linear_ws_bytes(1, 2048, 4096, 4096, 2) == 0  # enough tiles
+    assert L.bitnest_linear_ws_bytes(1, 1, 4096, 4096, 1) == 0  # the GEMV takes none
+    assert L.bitnest_linear_ws_bytes(3, 16, 300, 1024, 2) == -1
+    assert L.bitnest_linear_ws_bytes(1, 16, 300, 1000, 2) == -2
+    assert L.bitnest_linear_ws_bytes(1, 0, 300, 1024, 2) == 0
+    # automatic choice with scratch: the TMA-ring GEMV for 4 tokens; for 8
+    # tokens at K = 14336 (too many to stage for it) the split tensor-core path
+    assert L.bitnest_linear_ws_bytes(1, 4, 4096, 14336, 0) == 0
+    assert L.bitnest_linear_ws_bytes(1, 8, 4096, 14336, 0) > 0
+    assert bn.select_path(bn.TARGET, 8, 4096, 14336) == bn.PATH_GEMV  # without scratch
+
+    def call(ws=A, nbytes=need, M=16, N=300, K=1024, path=2):
+        return L.bitnest_linear_ws(1, v(A), v(A), v(A), v(A), v(A), v(A), M, N, K, v(A), 0,
+                                   None, path, v(ws) if ws else None, nbytes, None)
+
+    assert call(ws=0) == 1
+    assert call(nbytes=need - 16) == 1
+    assert call(ws=MIS) == 3
+    assert call(K=200) == 2
+    assert call(path=7) == 1
+    assert call(M=0) == 0

@@ -19,7 +19,7 @@ torch = pytest.importorskip("torch")
 if not torch.cuda.is_available():  # pragma: no cover
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from test_gpu_parity import Problem, dev, host  # noqa: E402
+from test_gpu_parity import DEV, Problem, dev, host  # noqa: E402
 
 
 @pytest.fixture(autouse=True)
@@ -122,3 +122,70 @@ def test_tc_persistent_tiles(mode, act_group):
         S = bn.debug_group_sums(mode, p.d_hi, p.d_lo, p.d_xq, p.d_xsum, path=bn.PATH_TC)
         torch.cuda.synchronize()
         assert np.array_equal(host(S), oracle.group_sums(mode, p.hi, p.lo, p.q, K))
+
+
+# ------------------------------------------------------------------ split K
+SPLIT_SHAPES = [(1, 100, 4096), (16, 300, 1024), (33, 129, 2048), (100, 1000, 1152),
+                (128, 256, 14336)]
+
+
+@pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("act_group", [0, 128])
+def test_tc_split_k_matches_oracle(M, N, K, mode, act_group):
+    """Too few (row tile, token tile) pairs to fill the GPU: the tensor-core
+    path splits K through the scratch (ragged K ranges, ragged tiles).  y
+    matches the oracle, and a second call on the same scratch (whose
+    counters the first left at zero) gives the same bits."""
+    p = Problem(M, N, K, seed=31 * M + N, act_group=act_group, bias=(M == 33))
+    nbytes = bn.linear_ws_bytes(mode, M, N, K, bn.PATH_TC)
+    assert nbytes > 0
+    ws = bn.workspace(nbytes, DEV)
+    args = (mode, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, p.d_xsum, ws, act_group, p.d_bias)
+    y1 = bn.linear_ws(*args, path=bn.PATH_TC)
+    y2 = bn.linear_ws(*args, path=bn.PATH_TC)
+    torch.cuda.synchronize()
+    assert oracle.max_normalised_error(host(y1), p.y_ref(mode)) <= TOL
+    assert torch.equal(y1, y2)
+    assert int(torch.count_nonzero(ws[-32:])) == 0  # the last tile's arrival counters
+
+
+def test_tc_split_k_llama3_down_proj_sampled():
+    """down_proj (N = 4096, K = 14336) at 16 and 128 tokens, where the split
+    applies: sampled rows against the oracle, and the unsplit call agrees."""
+    name = "down_proj"
+    N, K, act_group = synth.LLAMA3_8B_PROJECTIONS[name]
+    pid = synth.PROJ_IDS[name]
+    uh = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K)
+    ul = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K)
+    s = synth.group_scales(synth.SEED_SCALES + pid, N, K)
+    d_hi, d_lo = bn.pack_planes(dev(uh), dev(ul))
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 1],
+                                     np.random.default_rng(5).choice(N, 40, replace=False)]))
+    hi_r, lo_r = oracle.pack_plane(uh[rows]), oracle.pack_plane(ul[rows])
+    for M in (16, 128):
+        x = synth.activations(synth.SEED_ACTS + pid + M, M, K)
+        q, xs = oracle.quantize(x, act_group)
+        d_xq, d_xs, d_xsum = bn.quantize_act(dev(x), act_group)
+        for mode in (0, 1):
+            ws = bn.workspace(bn.linear_ws_bytes(mode, M, N, K, bn.PATH_TC), DEV)
+            y = bn.linear_ws(mode, d_hi, d_lo, dev(s), d_xq, d_xs, d_xsum, ws, act_group,
+                             path=bn.PATH_TC)
+            y0 = bn.linear(mode, d_hi, d_lo, dev(s), d_xq, d_xs, d_xsum, act_group,
+                           path=bn.PATH_TC)
+            torch.cuda.synchronize()
+            y_ref = oracle.linear(mode, hi_r, lo_r if mode else None, s[rows], q, xs, K,
+                                  act_group)
+            assert oracle.max_normalised_error(host(y)[:, rows], y_ref) <= TOL
+            assert oracle.max_normalised_error(host(y), host(y0).astype(np.float64)) <= TOL
+
+
+def test_tc_without_split_needs_no_scratch():
+    """Enough tiles: no scratch is needed and linear_ws is linear."""
+    M, N, K = 300, 2000, 256
+    assert bn.linear_ws_bytes(1, M, N, K, bn.PATH_TC) == 0
+    p = Problem(M, N, K, seed=5)
+    y = bn.linear_ws(1, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, p.d_xsum, None, path=bn.PATH_TC)
+    y0 = bn.linear(1, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, p.d_xsum, path=bn.PATH_TC)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0)

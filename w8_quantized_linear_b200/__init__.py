@@ -60,9 +60,12 @@ def lib() -> ctypes.CDLL:
     L.bitnest_select_path.argtypes = [I, I64, I64, I64]
     L.bitnest_debug_group_sums.argtypes = [I, P, P, P, P, I64, I64, I64, P, I, P]
     L.bitnest_quantize_linear.argtypes = [I, P, P, P, P, I64, I64, I64, P, I, P, P, P, P, I, P]
+    L.bitnest_linear_ws.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, I, P, I64, P]
+    L.bitnest_linear_ws_bytes.argtypes = [I, I64, I64, I64, I]
+    L.bitnest_linear_ws_bytes.restype = I64
     for name in ("bitnest_pack_planes", "bitnest_quantize_act", "bitnest_act_group_sums",
                  "bitnest_linear", "bitnest_linear_path", "bitnest_select_path",
-                 "bitnest_debug_group_sums", "bitnest_quantize_linear"):
+                 "bitnest_debug_group_sums", "bitnest_quantize_linear", "bitnest_linear_ws"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -151,6 +154,38 @@ def linear(mode: int, hi, lo, scale, xq, xscale, xsum, act_group: int = 0, bias=
     _check(lib().bitnest_linear_path(int(mode), _ptr(hi), _ptr(lo), _ptr(scale), _ptr(xq),
                                      _ptr(xscale), _ptr(xsum), M, N, K, _ptr(y), int(act_group),
                                      _ptr(bias), int(path), _stream(xq)), "bitnest_linear")
+    return y
+
+
+def linear_ws_bytes(mode: int, M: int, N: int, K: int, path: int = PATH_AUTO) -> int:
+    """Scratch bytes `linear_ws` uses for this problem (0: no split of K)."""
+    n = lib().bitnest_linear_ws_bytes(int(mode), int(M), int(N), int(K), int(path))
+    if n < 0:
+        _check(-n, "bitnest_linear_ws_bytes")
+    return n
+
+
+def workspace(nbytes: int, device):
+    """Zeroed scratch for `linear_ws` (its counters must start at zero)."""
+    import torch
+
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def linear_ws(mode: int, hi, lo, scale, xq, xscale, xsum, ws, act_group: int = 0, bias=None,
+              out=None, path: int = PATH_AUTO):
+    """`linear` with scratch `ws` (from `workspace`) that lets the tensor-core
+    path split K across CTAs when the layer has few output tiles."""
+    import torch
+
+    M, K = xq.shape
+    N = hi.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=xq.device)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().bitnest_linear_ws(int(mode), _ptr(hi), _ptr(lo), _ptr(scale), _ptr(xq),
+                                   _ptr(xscale), _ptr(xsum), M, N, K, _ptr(y), int(act_group),
+                                   _ptr(bias), int(path), _ptr(ws), nbytes, _stream(xq)),
+           "bitnest_linear_ws")
     return y
 
 

@@ -41,9 +41,13 @@ int check_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t 
   return BITNEST_OK;
 }
 
-int pick_path(int mode, int64_t M, int64_t N, int64_t K) {
+// The TMA-ring GEMV where it applies; with split-K scratch available, the
+// tensor-core path before the plain-load GEMV (whose single pass over a long
+// K with up to 8 tokens is slower than K split across the GPU).
+int pick_path(int mode, int64_t M, int64_t N, int64_t K, bool ws = false) {
   (void)mode;
-  (void)N;
+  if (gemv_tma_supported(M, N, K)) return BITNEST_PATH_GEMV;
+  if (ws && tc_ws_bytes(M, N, K) > 0) return BITNEST_PATH_TC;
   if (gemv_fits(M, K)) return BITNEST_PATH_GEMV;
   return BITNEST_PATH_TC;
 }
@@ -138,6 +142,41 @@ int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const ui
   if (M == 0 || N == 0) return BITNEST_OK;
   LinearArgs a{mode, hi, mode == BITNEST_TARGET ? lo : nullptr, scale, xq, xscale, xsum,
                bias, y, nullptr, M, N, K, act_group, overlap};
+  return run_linear(a, path, (cudaStream_t)stream);
+}
+
+int64_t bitnest_linear_ws_bytes(int mode, int64_t M, int64_t N, int64_t K, int path) {
+  path &= ~BITNEST_PATH_OVERLAP;
+  if (mode != BITNEST_DRAFT && mode != BITNEST_TARGET) return -BITNEST_ERR_INVALID_ARG;
+  if (path < BITNEST_PATH_AUTO || path > BITNEST_PATH_TC) return -BITNEST_ERR_INVALID_ARG;
+  if (check_shape(M, N, K) != BITNEST_OK) return -BITNEST_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return 0;
+  if (path == BITNEST_PATH_AUTO) path = pick_path(mode, M, N, K, true);
+  return path == BITNEST_PATH_TC ? tc_ws_bytes(M, N, K) : 0;
+}
+
+int bitnest_linear_ws(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                      const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
+                      int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
+                      int path, void *ws, int64_t ws_bytes, void *stream) {
+  const bool overlap = (path & BITNEST_PATH_OVERLAP) != 0;
+  path &= ~BITNEST_PATH_OVERLAP;
+  if (path < BITNEST_PATH_AUTO || path > BITNEST_PATH_TC) return BITNEST_ERR_INVALID_ARG;
+  int s = check_linear(mode, hi, lo, scale, xq, xscale, xsum, M, N, K, y, act_group, bias);
+  if (s != BITNEST_OK) return s;
+  if (M == 0 || N == 0) return BITNEST_OK;
+  if (path == BITNEST_PATH_AUTO) path = pick_path(mode, M, N, K, true);
+  const int64_t need = path == BITNEST_PATH_TC ? tc_ws_bytes(M, N, K) : 0;
+  if (need > 0) {
+    if (!ws || ws_bytes < need) return BITNEST_ERR_INVALID_ARG;
+    if (misaligned(ws)) return BITNEST_ERR_MISALIGNED;
+  }
+  LinearArgs a{mode, hi, mode == BITNEST_TARGET ? lo : nullptr, scale, xq, xscale, xsum,
+               bias, y, nullptr, M, N, K, act_group, overlap};
+  if (need > 0) {
+    a.ws = ws;
+    a.ws_bytes = ws_bytes;
+  }
   return run_linear(a, path, (cudaStream_t)stream);
 }
 

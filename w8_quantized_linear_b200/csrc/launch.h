@@ -20,6 +20,10 @@ struct LinearArgs {
   int64_t M, N, K;
   int act_group;          // 0 or 128
   bool overlap;           // launch with programmatic dependent launch
+  // scratch of the tensor-core path's split K (null: no split), its bytes;
+  // its counter area is zero before the call and zero again after it
+  void *ws = nullptr;
+  int64_t ws_bytes = 0;
 };
 
 cudaError_t launch_pack(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K, uint8_t *hi,
@@ -41,6 +45,8 @@ cudaError_t read_wait_timeout_gemv(int *flag, bool reset);
 // tcgen05 tensor-core GEMM (any M).
 bool tc_supported(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_tc(const LinearArgs &a, cudaStream_t st);
+// Scratch bytes the tensor-core path splits K with for this shape (0: none).
+int64_t tc_ws_bytes(int64_t M, int64_t N, int64_t K);
 
 // The flag a bounded wait sets when it gives up (synchronous read).
 cudaError_t read_wait_timeout(int *flag, bool reset);

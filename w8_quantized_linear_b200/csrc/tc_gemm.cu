@@ -63,11 +63,33 @@ struct Params {
   const uint16_t *bias;    // [N] or null
   float *y;                // [M, N]
   int32_t *S;              // debug sums [M, N, G]
+  // split K: each (row tile, token tile) is cut into `splits` ranges of `gps`
+  // groups; a range's partial sums go to ws, and the last of the splits to
+  // finish a warp's sub-block adds them (in split order) and writes y
+  float *ws;               // [row tiles x token tiles][splits][BW][BT] (splits > 1)
+  int *cnt;                // [row tiles x token tiles][kNumEpi] arrival counters, zero
   int M, N, K, G;
   int mt;                  // token tiles
-  int tiles;               // row tiles x token tiles
+  int splits, gps;         // K ranges per tile and groups per range
+  int tiles;               // row tiles x token tiles x splits
   int stages;
 };
+
+// Work item `tile`: its (row tile, token tile) index, K range and groups.
+struct TileCoord {
+  int tmn, split, n0, m0, g0, g1;
+};
+template <int BT>
+__device__ __forceinline__ TileCoord tile_coord(const Params &p, int tile) {
+  TileCoord c;
+  c.split = tile % p.splits;
+  c.tmn = tile / p.splits;
+  c.n0 = (c.tmn / p.mt) * BW;
+  c.m0 = (c.tmn % p.mt) * BT;
+  c.g0 = c.split * p.gps;
+  c.g1 = min(p.G, c.g0 + p.gps);
+  return c;
+}
 
 __host__ __device__ constexpr int tmem_cols(int bt) {
   // kAccBufs * bt rounded up to a power of two >= 32
@@ -147,7 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tslot = reinterpret_cast<uint32_t *>(accEmpty + kAccBufs);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = p.mt;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -187,7 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;  // stage slot and the parity of its current fill
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-      for (int g = 0; g < G; ++g) {
+      const TileCoord tc = tile_coord<BT>(p, tile);
+      for (int g = tc.g0; g < tc.g1; ++g) {
         ok = mbar_wait_warp(&fullB[s], ph);
         if (!ok) break;
         const uint8_t *hs = sH(s);
@@ -243,8 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       constexpr uint32_t bytes = BT * 128 + BW * 64 * (MODE ? 2 : 1);
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-        const int n0 = (tile / mt) * BW, m0 = (tile % mt) * BT;
-        for (int g = 0; g < G; ++g, ++it) {
+        const TileCoord tc = tile_coord<BT>(p, tile);
+        const int n0 = tc.n0, m0 = tc.m0;
+        for (int g = tc.g0; g < tc.g1; ++g, ++it) {
           if (!mbar_wait(&stageFree[s], ph ^ 1u)) {
             ok = false;
             break;
@@ -274,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint64_t kStageDesc = STAGE >> 4;  // descriptor address unit: 16 bytes
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-        for (int g = 0; g < G; ++g, ++it) {
+        const TileCoord tc = tile_coord<BT>(p, tile);
+        for (int g = tc.g0; g < tc.g1; ++g, ++it) {
           ok = mbar_wait(&fullB[s], ph) && mbar_wait(&fullA[s], ph) &&
                mbar_wait(&accEmpty[b], bph ^ 1u);
           if (!ok) break;
@@ -312,8 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-      const int n0 = (tile / mt) * BW, m0 = (tile % mt) * BT;
-      for (int gb = 0; gb < G && ok; gb += kCBatch) {
+      const TileCoord tc = tile_coord<BT>(p, tile);
+      const int n0 = tc.n0, m0 = tc.m0, G1 = tc.g1;
+      for (int gb = tc.g0; gb < G1 && ok; gb += kCBatch) {
         uint16_t sv[4][kCBatch];
         int rv[TU][kCBatch];
         float xv[TU][kCBatch];
@@ -322,8 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = n0 + lane + 32 * r;
 #pragma unroll
           for (int k = 0; k < kCBatch; ++k)
-            sv[r][k] = (!DEBUG && n < p.N && gb + k < G) ? __ldg(p.scale + (int64_t)n * G + gb + k)
-                                                          : (uint16_t)0;
+            sv[r][k] = (!DEBUG && n < p.N && gb + k < G1) ? __ldg(p.scale + (int64_t)n * G + gb + k)
+                                                           : (uint16_t)0;
         }
 #pragma unroll
         for (int u = 0; u < TU; ++u) {
@@ -331,14 +356,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool in = j < BT && m < p.M;
 #pragma unroll
           for (int k = 0; k < kCBatch; ++k) {
-            rv[u][k] = (in && gb + k < G) ? __ldg(p.xsum + (int64_t)m * G + gb + k) : 0;
-            xv[u][k] = (ACTG && in && gb + k < G) ? __ldg(p.xscale + (int64_t)m * G + gb + k)
-                                                  : 0.0f;
+            rv[u][k] = (in && gb + k < G1) ? __ldg(p.xsum + (int64_t)m * G + gb + k) : 0;
+            xv[u][k] = (ACTG && in && gb + k < G1) ? __ldg(p.xscale + (int64_t)m * G + gb + k)
+                                                   : 0.0f;
           }
         }
 #pragma unroll
         for (int k = 0; k < kCBatch; ++k) {
-          if (gb + k >= G) break;
+          if (gb + k >= G1) break;
           const int c = it % kCSlots;
           ok = mbar_wait_warp(&emptyC[c], ((it / kCSlots) & 1) ^ 1);
           if (!ok) break;
@@ -373,11 +398,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-      const int n = (tile / mt) * BW + row, m0 = (tile % mt) * BT;
+      const TileCoord tc = tile_coord<BT>(p, tile);
+      const int n = tc.n0 + row, m0 = tc.m0;
       float acc[COLS];
 #pragma unroll
       for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
-      for (int g = 0; g < G; ++g, ++it) {
+      for (int g = tc.g0; g < tc.g1; ++g, ++it) {
         const int cs = it % kCSlots, b = it % kAccBufs;
         ok = mbar_wait_warp(&fullC[cs], (it / kCSlots) & 1) &&
              mbar_wait_warp(&accFull[b], (it / kAccBufs) & 1);
@@ -425,6 +451,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           mbar_arrive(&accEmpty[b]);
           mbar_arrive(&emptyC[cs]);
+        }
+      }
+      if (!DEBUG && ok && p.splits > 1) {
+        // this range's partial sums of the warp's sub-block (rows of its lane
+        // quarter, its columns), then one arrival per warp; the last of the
+        // splits to arrive adds them all in split order
+        float *part = p.ws + ((int64_t)tc.tmn * p.splits) * (BW * BT) + row * BT + col0;
+#pragma unroll
+        for (int j = 0; j < COLS; j += 4)
+          *reinterpret_cast<float4 *>(part + (int64_t)tc.split * (BW * BT) + j) =
+              make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = atomicAdd(&p.cnt[tc.tmn * kNumEpi + e], 1) == p.splits - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        __threadfence();
+        if (lane == 0) p.cnt[tc.tmn * kNumEpi + e] = 0;  // ready for the next call
+#pragma unroll
+        for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
+        for (int sp = 0; sp < p.splits; ++sp) {
+#pragma unroll
+          for (int j = 0; j < COLS; j += 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(part + (int64_t)sp * (BW * BT) + j));
+            acc[j] += v.x;
+            acc[j + 1] += v.y;
+            acc[j + 2] += v.z;
+            acc[j + 3] += v.w;
+          }
         }
       }
       if (!DEBUG && ok && n < p.N) {
@@ -503,6 +559,36 @@ int num_sms() {
   return sms[dev] > 0 ? sms[dev] : 148;
 }
 
+// Split-K plan of a shape: a (row tile, token tile) grid that fills fewer
+// than half of the SMs is cut along K into ranges of at least four groups,
+// about one work item per SM in all.  Bytes: the partial tiles, then one
+// arrival counter per epilogue warp and tile (16-byte aligned).
+struct SplitPlan {
+  int splits, gps;
+  int64_t tmn, part_bytes, bytes;
+};
+SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int bt) {
+  SplitPlan sp;
+  const int G = (int)(K / kGroup);
+  sp.tmn = ((N + BW - 1) / BW) * ((M + bt - 1) / bt);
+  const int sms = num_sms();
+  int s = 1;
+  if (sp.tmn * 2 <= sms) {
+    s = (int)(sms / sp.tmn);
+    if (s > G / 4) s = G / 4;
+    if (s < 1) s = 1;
+  }
+  sp.gps = (G + s - 1) / s;
+  sp.splits = (G + sp.gps - 1) / sp.gps;  // no empty range
+  if (sp.splits == 1) {
+    sp.part_bytes = sp.bytes = 0;
+    return sp;
+  }
+  sp.part_bytes = sp.tmn * sp.splits * BW * bt * 4;
+  sp.bytes = sp.part_bytes + (sp.tmn * kNumEpi * 4 + 15) / 16 * 16;
+  return sp;
+}
+
 template <int MODE, int BT, bool ACTG, bool DEBUG>
 cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   const int G = (int)(a.K / kGroup);
@@ -531,7 +617,21 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   p.K = (int)a.K;
   p.G = G;
   p.mt = (int)((a.M + BT - 1) / BT);
-  const int64_t tiles = ((a.N + BW - 1) / BW) * (int64_t)p.mt;
+  p.splits = 1;
+  p.gps = G;
+  p.ws = nullptr;
+  p.cnt = nullptr;
+  if (a.ws && !DEBUG) {
+    const SplitPlan sp = split_plan(a.M, a.N, a.K, BT);
+    if (sp.splits > 1) {
+      if (a.ws_bytes < sp.bytes) return cudaErrorInvalidValue;
+      p.splits = sp.splits;
+      p.gps = sp.gps;
+      p.ws = static_cast<float *>(a.ws);
+      p.cnt = reinterpret_cast<int *>(static_cast<uint8_t *>(a.ws) + sp.part_bytes);
+    }
+  }
+  const int64_t tiles = ((a.N + BW - 1) / BW) * (int64_t)p.mt * p.splits;
   if (tiles > (1 << 30)) return cudaErrorInvalidValue;
   p.tiles = (int)tiles;
   p.stages = stages;
@@ -548,7 +648,10 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
 
 template <int MODE, int BT, bool DEBUG>
 cudaError_t launch_g(const LinearArgs &a, cudaStream_t st) {
-  if (a.act_group != 0 && !DEBUG) return launch_t<MODE, BT, true, DEBUG>(a, st);
+  // the debug sums take no activation scale: no per-group scale variant
+  if constexpr (!DEBUG) {
+    if (a.act_group != 0) return launch_t<MODE, BT, true, false>(a, st);
+  }
   return launch_t<MODE, BT, false, DEBUG>(a, st);
 }
 
@@ -575,6 +678,11 @@ bool tc_supported(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || M > (int64_t)1 << 30 || N > (int64_t)1 << 30) return false;
   if (K < kGroup || K % kGroup != 0 || K > ((int64_t)1 << 30)) return false;
   return tc::pick_stages(1, tc::pick_bt(M), tc::kMaxSmem) >= 2;
+}
+
+int64_t tc_ws_bytes(int64_t M, int64_t N, int64_t K) {
+  if (!tc_supported(M, N, K)) return 0;
+  return tc::split_plan(M, N, K, tc::pick_bt(M)).bytes;
 }
 
 cudaError_t launch_tc(const LinearArgs &a, cudaStream_t st) {
