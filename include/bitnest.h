@@ -164,9 +164,10 @@ int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const ui
  *   ws, ws_bytes : at least bitnest_linear_ws_bytes(mode, M, N, K, path)
  *                  bytes (BITNEST_ERR_INVALID_ARG if fewer).  When that is 0
  *                  ws may be NULL and the call is bitnest_linear_path.
- * The tail of ws holds arrival counters that must be zero before the first
- * call (cudaMemset once); every call leaves them zero.  Calls sharing one ws
- * must not run at the same time (calls in order on one stream are fine).
+ * The first 8 KB of ws hold arrival counters that must be zero before the
+ * first call (cudaMemset once); every call leaves them zero, so one ws can
+ * serve calls of any shapes.  Calls sharing one ws must not run at the same
+ * time (calls in order on one stream are fine).
  * With BITNEST_PATH_AUTO the choice may differ from bitnest_select_path's:
  * where the TMA-ring GEMV does not apply and K would be split, the
  * tensor-core path is taken (e.g. 5..8 tokens with K = 14336).

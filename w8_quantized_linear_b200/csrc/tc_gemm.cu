@@ -68,6 +68,7 @@ struct Params {
   // finish a warp's sub-block adds them (in split order) and writes y
   float *ws;               // [row tiles x token tiles][splits][BW][BT] (splits > 1)
   int *cnt;                // [row tiles x token tiles][kNumEpi] arrival counters, zero
+                           // (at the start of the scratch, ws after them)
   int M, N, K, G;
   int mt;                  // token tiles
   int splits, gps;         // K ranges per tile and groups per range
@@ -561,11 +562,15 @@ int num_sms() {
 
 // Split-K plan of a shape: a (row tile, token tile) grid that fills fewer
 // than half of the SMs is cut along K into ranges of at least four groups,
-// about one work item per SM in all.  Bytes: the partial tiles, then one
-// arrival counter per epilogue warp and tile (16-byte aligned).
+// about one work item per SM in all.  Scratch: the arrival counters (one
+// per epilogue warp and tile) at a fixed place, the start, so that calls of
+// any shapes can share one scratch (each leaves its counters zero, and no
+// shape's partial tiles reach another's counters); then the partial tiles.
+constexpr int kMaxCntTiles = 256;
+constexpr int64_t kCntBytes = int64_t(kMaxCntTiles) * kNumEpi * 4;  // 8 KB
 struct SplitPlan {
   int splits, gps;
-  int64_t tmn, part_bytes, bytes;
+  int64_t tmn, bytes;
 };
 SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int bt) {
   SplitPlan sp;
@@ -573,19 +578,14 @@ SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int bt) {
   sp.tmn = ((N + BW - 1) / BW) * ((M + bt - 1) / bt);
   const int sms = num_sms();
   int s = 1;
-  if (sp.tmn * 2 <= sms) {
+  if (sp.tmn * 2 <= sms && sp.tmn <= kMaxCntTiles) {
     s = (int)(sms / sp.tmn);
     if (s > G / 4) s = G / 4;
     if (s < 1) s = 1;
   }
   sp.gps = (G + s - 1) / s;
   sp.splits = (G + sp.gps - 1) / sp.gps;  // no empty range
-  if (sp.splits == 1) {
-    sp.part_bytes = sp.bytes = 0;
-    return sp;
-  }
-  sp.part_bytes = sp.tmn * sp.splits * BW * bt * 4;
-  sp.bytes = sp.part_bytes + (sp.tmn * kNumEpi * 4 + 15) / 16 * 16;
+  sp.bytes = sp.splits == 1 ? 0 : kCntBytes + sp.tmn * sp.splits * BW * bt * 4;
   return sp;
 }
 
@@ -627,8 +627,8 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
       if (a.ws_bytes < sp.bytes) return cudaErrorInvalidValue;
       p.splits = sp.splits;
       p.gps = sp.gps;
-      p.ws = static_cast<float *>(a.ws);
-      p.cnt = reinterpret_cast<int *>(static_cast<uint8_t *>(a.ws) + sp.part_bytes);
+      p.cnt = static_cast<int *>(a.ws);
+      p.ws = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + kCntBytes);
     }
   }
   const int64_t tiles = ((a.N + BW - 1) / BW) * (int64_t)p.mt * p.splits;
