@@ -178,6 +178,31 @@ int bitnest_linear_ws(int mode, const uint8_t *hi, const uint8_t *lo, const uint
                       int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,
                       int path, void *ws, int64_t ws_bytes, void *stream);
 
+/*
+ * bitnest_linear_ws without caller scratch and without any allocation: the
+ * split-K partial sums and counters live in one file-scope static device
+ * array of the library, BITNEST_STATIC_WS_BYTES (12 MiB) per device, zero
+ * from module load and left zero by every call.  (The BitNest pages have no
+ * counterpart to this entry point: it is a deployment convenience of this
+ * library.)  The library calls no cudaMalloc / cudaFree here; it looks up the
+ * array's device address once per device (cudaGetSymbolAddress) and caches it.
+ *   - A problem whose split needs more than BITNEST_STATIC_WS_BYTES returns
+ *     BITNEST_ERR_UNSUPPORTED_SHAPE, launching nothing.
+ *   - Every call on a device shares the one array: calls that overlap in
+ *     time (on different streams or threads) race and give wrong results.
+ *     Calls in order on one stream are safe, BITNEST_PATH_OVERLAP included.
+ *   - Make the first call on each device outside CUDA stream capture (the
+ *     address lookup is not a capturable operation); later calls may be
+ *     captured.
+ * Results are bit-identical to bitnest_linear_ws's for the same arguments.
+ * Other arguments, checks and errors: as bitnest_linear_ws.
+ */
+#define BITNEST_STATIC_WS_BYTES (12LL << 20)
+int bitnest_linear_static_ws(int mode, const uint8_t *hi, const uint8_t *lo,
+                             const uint16_t *scale, const int8_t *xq, const float *xscale,
+                             const int32_t *xsum, int64_t M, int64_t N, int64_t K, float *y,
+                             int act_group, const uint16_t *bias, int path, void *stream);
+
 /* Scratch bytes bitnest_linear_ws uses for this problem and path (0 when the
  * path does not split K).  Host only; -BITNEST_ERR_INVALID_ARG for a bad
  * mode or path, -BITNEST_ERR_UNSUPPORTED_SHAPE for a bad shape. */

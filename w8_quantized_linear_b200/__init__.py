@@ -61,11 +61,13 @@ def lib() -> ctypes.CDLL:
     L.bitnest_debug_group_sums.argtypes = [I, P, P, P, P, I64, I64, I64, P, I, P]
     L.bitnest_quantize_linear.argtypes = [I, P, P, P, P, I64, I64, I64, P, I, P, P, P, P, I, P]
     L.bitnest_linear_ws.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, I, P, I64, P]
+    L.bitnest_linear_static_ws.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, I, P]
     L.bitnest_linear_ws_bytes.argtypes = [I, I64, I64, I64, I]
     L.bitnest_linear_ws_bytes.restype = I64
     for name in ("bitnest_pack_planes", "bitnest_quantize_act", "bitnest_act_group_sums",
                  "bitnest_linear", "bitnest_linear_path", "bitnest_select_path",
-                 "bitnest_debug_group_sums", "bitnest_quantize_linear", "bitnest_linear_ws"):
+                 "bitnest_debug_group_sums", "bitnest_quantize_linear", "bitnest_linear_ws",
+                 "bitnest_linear_static_ws"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -186,6 +188,22 @@ def linear_ws(mode: int, hi, lo, scale, xq, xscale, xsum, ws, act_group: int = 0
                                    _ptr(xscale), _ptr(xsum), M, N, K, _ptr(y), int(act_group),
                                    _ptr(bias), int(path), _ptr(ws), nbytes, _stream(xq)),
            "bitnest_linear_ws")
+    return y
+
+
+def linear_static_ws(mode: int, hi, lo, scale, xq, xscale, xsum, act_group: int = 0,
+                     bias=None, out=None, path: int = PATH_AUTO):
+    """`linear_ws` on the library's own static device scratch (no allocation;
+    calls that overlap in time race: see bitnest_linear_static_ws)."""
+    import torch
+
+    M, K = xq.shape
+    N = hi.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=xq.device)
+    _check(lib().bitnest_linear_static_ws(int(mode), _ptr(hi), _ptr(lo), _ptr(scale), _ptr(xq),
+                                          _ptr(xscale), _ptr(xsum), M, N, K, _ptr(y),
+                                          int(act_group), _ptr(bias), int(path), _stream(xq)),
+           "bitnest_linear_static_ws")
     return y
 
 

@@ -180,6 +180,31 @@ int bitnest_linear_ws(int mode, const uint8_t *hi, const uint8_t *lo, const uint
   return run_linear(a, path, (cudaStream_t)stream);
 }
 
+int bitnest_linear_static_ws(int mode, const uint8_t *hi, const uint8_t *lo,
+                             const uint16_t *scale, const int8_t *xq, const float *xscale,
+                             const int32_t *xsum, int64_t M, int64_t N, int64_t K, float *y,
+                             int act_group, const uint16_t *bias, int path, void *stream) {
+  static_assert(kStaticWsBytes == BITNEST_STATIC_WS_BYTES, "scratch size");
+  const bool overlap = (path & BITNEST_PATH_OVERLAP) != 0;
+  path &= ~BITNEST_PATH_OVERLAP;
+  if (path < BITNEST_PATH_AUTO || path > BITNEST_PATH_TC) return BITNEST_ERR_INVALID_ARG;
+  int s = check_linear(mode, hi, lo, scale, xq, xscale, xsum, M, N, K, y, act_group, bias);
+  if (s != BITNEST_OK) return s;
+  if (M == 0 || N == 0) return BITNEST_OK;
+  if (path == BITNEST_PATH_AUTO) path = pick_path(mode, M, N, K, true);
+  const int64_t need = path == BITNEST_PATH_TC ? tc_ws_bytes(M, N, K) : 0;
+  if (need > kStaticWsBytes) return BITNEST_ERR_UNSUPPORTED_SHAPE;
+  LinearArgs a{mode, hi, mode == BITNEST_TARGET ? lo : nullptr, scale, xq, xscale, xsum,
+               bias, y, nullptr, M, N, K, act_group, overlap};
+  if (need > 0) {
+    void *ws = nullptr;
+    if (tc_static_ws(&ws) != cudaSuccess) return BITNEST_ERR_CUDA;
+    a.ws = ws;
+    a.ws_bytes = kStaticWsBytes;
+  }
+  return run_linear(a, path, (cudaStream_t)stream);
+}
+
 int bitnest_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
                    const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
                    int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,

@@ -47,6 +47,10 @@ bool tc_supported(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_tc(const LinearArgs &a, cudaStream_t st);
 // Scratch bytes the tensor-core path splits K with for this shape (0: none).
 int64_t tc_ws_bytes(int64_t M, int64_t N, int64_t K);
+// Size and device address (looked up once per device) of the library's own
+// static split-K scratch.
+constexpr int64_t kStaticWsBytes = int64_t(12) << 20;
+cudaError_t tc_static_ws(void **ws);
 
 // The flag a bounded wait sets when it gives up (synchronous read).
 cudaError_t read_wait_timeout(int *flag, bool reset);

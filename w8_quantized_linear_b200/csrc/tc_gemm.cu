@@ -680,6 +680,29 @@ bool tc_supported(int64_t M, int64_t N, int64_t K) {
   return tc::pick_stages(1, tc::pick_bt(M), tc::kMaxSmem) >= 2;
 }
 
+// Library-owned split-K scratch for bitnest_linear_static_ws: zero at module
+// load (so its arrival counters start at zero) and left zero by every call.
+// The largest split plan is one 128 x 128 fp32 partial tile per SM plus the
+// counters: under 10 MB on 148 SMs.
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+
+cudaError_t tc_static_ws(void **ws) {
+  static void *addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!addr[dev]) {  // once per device
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_ws);
+    if (e != cudaSuccess) return e;
+    if (!p) return cudaErrorInvalidSymbol;
+    addr[dev] = p;
+  }
+  *ws = addr[dev];
+  return cudaSuccess;
+}
+
 int64_t tc_ws_bytes(int64_t M, int64_t N, int64_t K) {
   if (!tc_supported(M, N, K)) return 0;
   return tc::split_plan(M, N, K, tc::pick_bt(M)).bytes;
