@@ -699,16 +699,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=device)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = dist_helpers(world, device)
 
     wl = DecodeWorkload(device, overlap=not args.no_overlap)
     step_bytes = wl.step_bytes()
@@ -760,20 +751,9 @@ def main():
         "vs_baseline": None,
         "dtype": "int8 x u8/u4 -> int32, fp32 epilogue",
         "data": "synthetic (seeded SplitMix64: uniform nibbles, fp16 scales, N(0,1) activations with 4 x20 outliers)",
-        "config": {
-            "workload": wl_name,
-            "projections": {k: list(v[:2]) for k, v in synth.LLAMA3_8B_PROJECTIONS.items()},
-            "launches": "per pass: one quantise + linear kernel for q|k|v (fused, N=6144), o (per-group "
-                        "activation scales), gate|up (fused, N=28672), down",
-            "passes": "draft W4A8 M=1 then verify W8A8 M=4 (gamma+1)",
-            "group": 128,
-            "bytes_per_step": step_bytes,
-            "l2": f"inputs larger than L2: {N_COPIES} rotating copies of the layer weights "
-                  f"({N_COPIES * sum(v[0] * v[1] for v in synth.LLAMA3_8B_PROJECTIONS.values()) / 1e6:.0f} MB of planes)",
-            "parallelism": "replicas" if world > 1 else "single",
-            "timing": ("direct launches" if args.no_graph else "CUDA graph per step")
-                      + ", CUDA events on the launching stream",
-        },
+        "config": step_config(wl_name, world),
+        "timing": ("direct launches" if args.no_graph else "CUDA graph per step")
+                  + ", CUDA events on the launching stream, max over ranks",
         "clocks": clocks.summary(),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
@@ -803,6 +783,43 @@ def main():
         print(json.dumps(out), flush=True)
 
 
+def step_config(wl_name, world):
+    """The workload of one step (the same for both arms)."""
+    return {
+        "workload": wl_name,
+        "projections": {k: list(v[:2]) for k, v in synth.LLAMA3_8B_PROJECTIONS.items()},
+        "launches": "per pass: one quantise + linear call for q|k|v (fused, N=6144), o (per-group "
+                    "activation scales), gate|up (fused, N=28672), down",
+        "passes": "draft W4A8 M=1 then verify W8A8 M=4 (gamma+1)",
+        "group": 128,
+        "bytes_per_step": decode_step_bytes(),
+        "l2": f"inputs larger than L2: {N_COPIES} rotating copies of the layer weights "
+              f"({N_COPIES * sum(v[0] * v[1] for v in synth.LLAMA3_8B_PROJECTIONS.values()) / 1e6:.0f}"
+              " MB of planes)",
+        "parallelism": "replicas" if world > 1 else "single",
+    }
+
+
+def dist_helpers(world, device):
+    """barrier() and max_over_ranks(v) over the default process group (any
+    backend: CUDA tensors for nccl, CPU tensors for gloo); no-ops alone."""
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
 def run_reference(args, rank, world, wl_name):
     """The oracle, as it stands, on the host cores (rank 0 only)."""
     if rank != 0:
@@ -822,7 +839,8 @@ def run_reference(args, rank, world, wl_name):
         "steps": len(times), "warmup": args.warmup, "ms_per_step": round(1e3 * t, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int64 sums, fp64 output", "data": "synthetic",
-        "config": {"workload": wl_name},
+        "config": step_config(wl_name, world),
+        "timing": "host wall clock of the oracle, median over the steps",
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"first {rows} output rows of every projection and pass, "
