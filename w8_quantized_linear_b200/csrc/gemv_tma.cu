@@ -50,6 +50,10 @@ constexpr int kSegs = kStepCols / 256;                 // 128-byte plane segment
 constexpr int kPlaneBytes = kRows * kStepCols / 2;     // 32 KB: one TMA box per plane
 constexpr int kMaxStages = 8;
 constexpr int kRedSlots = 4;  // row blocks whose partial sums can be in flight
+// Weight stages the producer issues before the activations are loaded: the
+// stream starts while the preceding kernel runs, yet the memory queues are
+// short again when the consumers' activation loads go out.
+constexpr int kPreStages = 2;
 constexpr int kScaleSmemMax = 32 * 1024;  // the CTA's group scales are staged once
 constexpr int kSmemBudget = 227 * 1024;
 
@@ -85,7 +89,7 @@ __host__ __device__ inline int fixed_bytes(int M, int K, bool actg, int nb) {
 
 __host__ inline int smem_total(int mode, int M, bool actg, int K, int nb, int stages) {
   return 1024 + fixed_bytes(M, K, actg, nb) + stages * stage_bytes(mode) +
-         (2 * kMaxStages + 2 * kRedSlots) * 8;
+         (2 * kMaxStages + 2 * kRedSlots + 1) * 8;
 }
 
 // D = A (16x32 u8) * B (32x8 s8) + C, int32.  Not volatile: a pure function
@@ -153,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *empty = full + kMaxStages;
   uint64_t *part_full = empty + kMaxStages;       // [kRedSlots]: all warps' partials written
   uint64_t *slot_free = part_full + kRedSlots;    // [kRedSlots]: partials read out
+  uint64_t *act_issued = slot_free + kRedSlots;   // every consumer warp issued its activation loads
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -165,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&part_full[i], kConsumerWarps);
       mbar_init(&slot_free[i], 1);
     }
+    mbar_init(act_issued, kConsumerWarps);
     fence_barrier_init();
   }
   __syncthreads();
@@ -227,6 +233,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row0 = ((int)blockIdx.x + k * (int)gridDim.x) * kRows;
         for (int ks = 0; ks < p.nks; ++ks, ++it) {
           const int s = it % S;
+          // the rest of the stream queues behind the activation loads
+          if (it == kPreStages && !mbar_wait(act_issued, 0)) {
+            ok = false;
+            break;
+          }
           if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
             ok = false;
             break;
@@ -291,6 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool in = i < Gp * 8 && m < M && g < G;
       rv[u] = in ? __ldg(p.xsum + m * G + g) : 0;
       xv[u] = (ACTG && in) ? __ldg(p.xscale + m * G + g) : 0.0f;
+    }
+    if (bx == 0) {  // loads of the first batch issued: the weight stream may go on
+      __syncwarp();
+      if (lane == 0) mbar_arrive(act_issued);
     }
 #pragma unroll
     for (int u = 0; u < XB; ++u) {
