@@ -84,7 +84,8 @@ def test_pack_planes_bit_exact(N, K):
 
 
 @pytest.mark.parametrize("M,K", [(1, 128), (1, 4096), (4, 14336), (5, 1152), (33, 1024),
-                                 (129, 256), (2048, 4096)])
+                                 (129, 256), (2048, 4096), (16, 2048), (2, 1024), (3, 768),
+                                 (7, 512)])
 @pytest.mark.parametrize("act_group", [0, 128])
 def test_quantize_bit_exact(M, K, act_group):
     x = synth.activations(3100 + M, M, K)
