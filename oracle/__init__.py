@@ -59,6 +59,9 @@ def _load():
     lib.oracle_num_threads.restype = I
     lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
     lib.oracle_half_to_double.restype = ctypes.c_double
+    lib.oracle_float_to_half.argtypes = [ctypes.c_float]
+    lib.oracle_float_to_half.restype = ctypes.c_uint16
+    lib.oracle_pack_weights.argtypes = [P, I64, I64, P, P, P]
     lib.oracle_pack_plane.argtypes = [P, I64, I64, P]
     lib.oracle_unpack_plane.argtypes = [P, I64, I64, P]
     lib.oracle_dequant.argtypes = [I, P, P, P, I64, I64, P]
@@ -95,6 +98,27 @@ def num_threads() -> int:
 
 def half_to_double(bits: int) -> float:
     return float(_load().oracle_half_to_double(int(bits) & 0xFFFF))
+
+
+def float_to_half_bits(f) -> np.ndarray:
+    """fp32 values -> fp16 bit patterns (round to nearest, ties to even)."""
+    f = np.ascontiguousarray(np.asarray(f, np.float32))
+    lib = _load()
+    out = np.array([lib.oracle_float_to_half(float(v)) for v in f.ravel()], np.uint16)
+    return out.reshape(f.shape)
+
+
+def pack_weights(w):
+    """fp16 weights [N, K] -> (uh uint8 [N, K], ul uint8 [N, K], scale fp16
+    bits [N, K/128]): round-to-nearest 4-bit high nibble with scale
+    max|W| / 7 per row and group, closed-form residual low nibble."""
+    wb = _half_bits(w)
+    N, K = wb.shape
+    uh = np.empty((N, K), np.uint8)
+    ul = np.empty((N, K), np.uint8)
+    sc = np.empty((N, K // GROUP), np.uint16)
+    _load().oracle_pack_weights(_ptr(wb), N, K, _ptr(uh), _ptr(ul), _ptr(sc))
+    return uh, ul, sc
 
 
 def pack_plane(u: np.ndarray) -> np.ndarray:

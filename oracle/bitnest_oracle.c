@@ -64,6 +64,37 @@ double oracle_half_to_double(uint16_t h) {
 
 float oracle_half_to_float(uint16_t h) { return (float)oracle_half_to_double(h); }
 
+/* ---- fp16 encoding: binary32 -> binary16, round to nearest, ties to even --
+ * From the format's definition: the value is f = (-1)^s * m * 2^e with m an
+ * integer mantissa; binary16 keeps 11 significant bits for normal values
+ * (exponent -14 .. 15) and a fixed quantum of 2^-24 below 2^-14.  Rounding
+ * is done on the exact integer multiple of the target quantum, ties to even;
+ * magnitudes that round to 2^16 or more become infinity.                */
+uint16_t oracle_float_to_half(float f) {
+  uint32_t bits;
+  memcpy(&bits, &f, 4);
+  uint16_t sign = (uint16_t)((bits >> 16) & 0x8000u);
+  if (isnan(f)) return (uint16_t)(sign | 0x7e00u);
+  double a = fabs((double)f);
+  if (isinf(f) || a >= 65520.0) return (uint16_t)(sign | 0x7c00u); /* 65520 = 65504 + half a quantum */
+  if (a == 0.0) return sign;
+  int e2;
+  frexp(a, &e2);           /* a = fr * 2^e2 with fr in [0.5, 1) */
+  int exp = e2 - 1;        /* a in [2^exp, 2^(exp+1)) */
+  if (exp < -14) exp = -14; /* subnormal range: quantum 2^-24 */
+  double quantum = ldexp(1.0, exp - 10);
+  double mult = a / quantum; /* exact: a is a binary32 value */
+  double r = nearbyint(mult); /* default rounding mode: to nearest, ties to even */
+  uint32_t m = (uint32_t)r;
+  if (m == 2048) { /* rounded up to the next power of two */
+    m = 1024;
+    exp += 1;
+  }
+  if (m < 1024) return (uint16_t)(sign | m); /* subnormal (exp == -14) */
+  if (exp > 15) return (uint16_t)(sign | 0x7c00u);
+  return (uint16_t)(sign | ((uint32_t)(exp + 15) << 10) | (m - 1024));
+}
+
 /* ---- plane packing (model card, "Files": byte j = col 2j | col 2j+1 << 4) */
 void oracle_pack_plane(const uint8_t *u, int64_t N, int64_t K, uint8_t *plane) {
   for (int64_t n = 0; n < N; ++n)
@@ -113,6 +144,51 @@ void oracle_dequant(int mode, const uint8_t *hi, const uint8_t *lo, const uint16
       } else {
         int l = nibble(lo, K, n, k);
         W[n * K + k] = (double)(16 * (h - 8) + (l - 8)) * s / 16.0;
+      }
+    }
+}
+
+/* ---- packer from fp weights ----------------------------------------------
+ * Model card, opening paragraph: the high nibble is a 4-bit model fitted
+ * first, the low nibble the closed-form residual back to 8 bits; section
+ * "Files": u = q + 8, one fp16 scale per row and 128-column group, draft
+ * W4 = (hi - 8) * scale, target W8 = (16 (hi - 8) + (lo - 8)) * scale / 16.
+ * Readings (the card is silent on them; its GPTQ fit of the high nibble is
+ * not reproduced):
+ *   scale   s = fp16(max|W| / 7)   (the fp32 quotient rounded to fp16);
+ *   high    q4 = rne(t), t = W / s (one correctly rounded fp32 division);
+ *           |t| <= 7 (1 + 2^-10) keeps q4 in [-7, 7]: symmetric, no clamp;
+ *   low     ql = clamp(rne(16 (t - q4)), -8, 7)   (t - q4 is exact);
+ *   an all-zero group gets s = 0 and q4 = ql = 0.
+ * Outputs the unpacked nibbles uh = q4 + 8, ul = ql + 8 [N, K] and the fp16
+ * scale bits [N, K/128].                                                */
+void oracle_pack_weights(const uint16_t *w, int64_t N, int64_t K, uint8_t *uh, uint8_t *ul,
+                         uint16_t *scale) {
+  int64_t G = K / ORACLE_GROUP;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t g = 0; g < G; ++g) {
+      const uint16_t *wr = w + n * K + g * ORACLE_GROUP;
+      float amax = 0.0f;
+      for (int64_t k = 0; k < ORACLE_GROUP; ++k) {
+        float a = fabsf(oracle_half_to_float(wr[k]));
+        if (a > amax) amax = a;
+      }
+      uint16_t sbits = oracle_float_to_half(amax / 7.0f);
+      float s = oracle_half_to_float(sbits);
+      scale[n * G + g] = sbits;
+      for (int64_t k = 0; k < ORACLE_GROUP; ++k) {
+        int q4 = 0, ql = 0;
+        if (s != 0.0f) {
+          float t = oracle_half_to_float(wr[k]) / s;
+          float r4 = nearbyintf(t);
+          q4 = (int)r4;
+          float rl = nearbyintf(16.0f * (t - r4));
+          if (rl > 7.0f) rl = 7.0f;
+          if (rl < -8.0f) rl = -8.0f;
+          ql = (int)rl;
+        }
+        uh[n * K + g * ORACLE_GROUP + k] = (uint8_t)(q4 + 8);
+        ul[n * K + g * ORACLE_GROUP + k] = (uint8_t)(ql + 8);
       }
     }
 }

@@ -328,3 +328,98 @@ def test_normalised_error_metric():
     y = y_ref + np.array([0, 0, 1e-3 * 1e-3 * rms, 0])
     assert oracle.max_normalised_error(y, y_ref) == pytest.approx(1e-3, rel=1e-9)
     assert oracle.max_normalised_error(y_ref, y_ref) == 0.0
+
+
+# ------------------------------------------------------- fp16 encoding
+def test_float_to_half_exhaustive_round_trip(oracle_mod):
+    """Every finite fp16 value, widened to fp32, encodes back to itself."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    bits = bits[(bits & 0x7C00) != 0x7C00]
+    f32 = bits.view(np.float16).astype(np.float32)
+    assert np.array_equal(oracle_mod.float_to_half_bits(f32), bits)
+
+
+def test_float_to_half_matches_numpy(oracle_mod):
+    """Rounding (ties to even, subnormals, overflow) against numpy's fp16 cast."""
+    rng = np.random.default_rng(11)
+    mags = np.concatenate([10.0 ** rng.uniform(-9, 5, 4000), [65504, 65519.99, 65520, 70000,
+                                                              2.0 ** -25, 2.0 ** -24 * 1.5]])
+    f = (mags * rng.choice([-1, 1], mags.size)).astype(np.float32)
+    # exact midpoints between neighbouring fp16 values: ties go to the even one
+    h = rng.integers(0x0001, 0x7BFE, 500).astype(np.uint16)
+    lo = h.view(np.float16).astype(np.float64)
+    hi = (h + 1).view(np.float16).astype(np.float64)
+    f = np.concatenate([f, ((lo + hi) / 2).astype(np.float32)])
+    with np.errstate(over="ignore"):
+        ref = f.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle_mod.float_to_half_bits(f), ref)
+
+
+# -------------------------------------------------- packer from weights
+def _read_pack_cases():
+    cases, cur = [], None
+    with open(os.path.join(GOLDEN, "pack_weights_cases.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            tok = line.split()
+            if tok[0] == "case":
+                K = int(tok[2].split("=")[1])
+                cur = {"name": tok[1], "w": np.zeros(K), "uh": np.full(K, 8), "ul": np.full(K, 8)}
+                cases.append(cur)
+            elif tok[0] in ("w", "uh", "ul"):
+                for t in tok[1:]:
+                    i, v = t.split(":")
+                    cur[tok[0]][int(i)] = float(v)
+            elif tok[0] == "s":
+                cur["s"] = int(tok[1], 16)
+    return cases
+
+
+@pytest.mark.parametrize("case", _read_pack_cases(), ids=lambda c: c["name"])
+def test_pack_weights_golden(oracle_mod, case):
+    w = case["w"].astype(np.float16).reshape(1, -1)
+    assert np.array_equal(w.astype(np.float64)[0], case["w"])  # fixture exact in fp16
+    uh, ul, sc = oracle_mod.pack_weights(w)
+    assert uh[0].tolist() == case["uh"].astype(int).tolist()
+    assert ul[0].tolist() == case["ul"].astype(int).tolist()
+    assert int(sc[0, 0]) == case["s"]
+
+
+def test_pack_weights_recovers_codes_on_the_grid(oracle_mod):
+    """Weights exactly on the target grid (16 c4 + cl) s / 16, with the group
+    maximum 7 s: the packer returns those codes and that scale."""
+    rng = np.random.default_rng(3)
+    N, K = 6, 512
+    s = 2.0 ** -6
+    c4 = rng.integers(-6, 7, (N, K))
+    cl = rng.integers(-7, 8, (N, K))
+    c4[:, ::128] = rng.choice([-7, 7], (N, K // 128))  # one element at +-7 s per group
+    cl[:, ::128] = 0
+    w = ((16 * c4 + cl) * s / 16).astype(np.float16)
+    assert np.array_equal(w.astype(np.float64), (16 * c4 + cl) * s / 16)
+    uh, ul, sc = oracle_mod.pack_weights(w)
+    assert np.array_equal(uh.astype(int), c4 + 8)
+    assert np.array_equal(ul.astype(int), cl + 8)
+    assert np.all(sc == np.float16(s).view(np.uint16))
+
+
+def test_pack_weights_error_bounds(oracle_mod):
+    """Random weights: the draft is within s/2 of W, the target within s/16
+    (s/32 where the residual is not clipped), per element."""
+    rng = np.random.default_rng(4)
+    N, K = 8, 1024
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+    w[1, :128] = 0  # an all-zero group
+    uh, ul, sc = oracle_mod.pack_weights(w)
+    hi, lo = oracle_mod.pack_plane(uh), oracle_mod.pack_plane(ul)
+    W = w.astype(np.float64)
+    s = np.repeat(sc.view(np.float16).astype(np.float64), 128, axis=1)
+    d4 = np.abs(oracle_mod.dequant(0, hi, None, sc, K) - W)
+    d8 = np.abs(oracle_mod.dequant(1, hi, lo, sc, K) - W)
+    assert np.all(d4 <= s * 0.5 * (1 + 2.0 ** -20))
+    assert np.all(d8 <= s / 16 * (1 + 2.0 ** -20))
+    unclipped = ul < 15
+    assert np.all(d8[unclipped] <= s[unclipped] / 32 * (1 + 2.0 ** -20))
+    assert sc[1, 0] == 0 and np.all(uh[1, :128] == 8) and np.all(ul[1, :128] == 8)
