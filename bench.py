@@ -584,6 +584,47 @@ def measure_sweep(wl, hbm_peak, reps=5):
     return res
 
 
+# ------------------------------------------------ packer from fp weights
+def measure_pack(wl, hbm_peak, reps=5):
+    """bitnest_pack_weights on the seven projections' shapes (seeded
+    synthetic fp16 weights, N(0, 0.02^2)): one launch per projection after
+    a 256 MB L2 flush.  Bytes: fp16 weights read, both planes and the fp16
+    scales written."""
+    import torch
+
+    bn = wl.bn
+    dev = wl.dev
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(synth.SEED_WEIGHTS)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    res, tot_b, tot_t = {}, 0, 0.0
+    for name, (N, K, _) in wl.projs:
+        w = (torch.randn((N, K), generator=gen, device=dev, dtype=torch.float32) * 0.02).half()
+        out = bn.pack_weights(w)
+        t = 0.0
+        for _ in range(reps):
+            flush.fill_(1)
+            a.record()
+            bn.pack_weights(w, out=out)
+            b.record()
+            torch.cuda.synchronize()
+            t += a.elapsed_time(b) / 1e3
+        t /= reps
+        nbytes = 2 * N * K + N * K + 2 * N * (K // 128)
+        res[name] = {"us": round(t * 1e6, 2), "GB/s": round(nbytes / t / 1e9, 1),
+                     "frac_hbm": round(nbytes / t / 1e9 / hbm_peak, 3)}
+        tot_b += nbytes
+        tot_t += t
+        del w, out
+    del flush
+    return {"workload": "fp16 weights of the 7 Llama-3-8B-shaped projections -> planes + "
+                        "scales, one launch each after an L2 flush",
+            "GB/s": round(tot_b / tot_t / 1e9, 1), "frac_hbm": round(tot_b / tot_t / 1e9 / hbm_peak, 3),
+            "us_total": round(tot_t * 1e6, 1), "per_projection": res}
+
+
 # --------------------------------------------------------- decode round
 ROUND_LAYERS = 32
 ROUND_DRAFT_PASSES = 3  # gamma = 3 draft tokens, then one verify pass at M = gamma + 1
@@ -671,7 +712,7 @@ def main():
                     help="launch the step's kernels directly instead of replaying a CUDA graph "
                          "(for profilers that cannot replay the captured kernel nodes)")
     ap.add_argument("--workload", default="all",
-                    choices=["all", "decode", "prefill", "sweep", "round"],
+                    choices=["all", "decode", "prefill", "sweep", "round", "pack"],
                     help="all: the decode step line with the prefill, M-sweep and "
                          "decode-round objects; otherwise only that part (profiling runs)")
     args = ap.parse_args()
@@ -712,6 +753,9 @@ def main():
         sweep = measure_sweep(wl, hbm_peak, reps=5 if args.workload == "all" else 2)
     if args.workload in ("all", "round"):
         rnd = measure_round(wl, hbm_peak, reps=10 if args.workload == "all" else 3)
+    pack = None
+    if args.workload in ("all", "pack"):
+        pack = measure_pack(wl, hbm_peak)
     prefill = None
     if args.workload in ("all", "prefill"):
         pre, pre_ops, pre_t = measure_prefill(wl, reps=10 if args.workload == "all" else 3)
@@ -732,7 +776,8 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         if rank == 0:
-            part = {"prefill": prefill, "m_sweep": sweep, "decode_round": rnd}
+            part = {"prefill": prefill, "m_sweep": sweep, "decode_round": rnd,
+                    "pack_from_weights": pack}
             print(json.dumps({"metric": METRIC, "workload": f"{args.workload} only",
                               **{k: v for k, v in part.items() if v is not None}}), flush=True)
         return
@@ -769,6 +814,8 @@ def main():
                           "per_case": sweep}
     if rnd is not None:
         out["decode_round"] = rnd
+    if pack is not None:
+        out["pack_from_weights"] = pack
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, cores, rows = cpu_baseline()
         out["cpu_baseline"] = {

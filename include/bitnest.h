@@ -87,6 +87,28 @@ int bitnest_version(void);
 int bitnest_device_wait_timeout(int reset);
 
 /*
+ * Build the planes and scales of one layer from its fp16 weights
+ * (BitNest-Llama-3-8B model card, opening paragraph: the high nibble is a
+ * 4-bit model fitted first, the low nibble the closed-form residual back to
+ * 8 bits; section "Files": u = q + 8, one fp16 scale per 128 columns).  The
+ * card fits the high nibble with GPTQ, which needs calibration data; this
+ * packer rounds it to nearest instead:
+ *   s  = fp16(max|W| / 7) per row and 128-column group (0 for an all-zero
+ *        group, whose nibbles are then 8),
+ *   t  = W / s (fp32, correctly rounded),
+ *   hi = rne(t) + 8,  lo = clamp(rne(16 (t - (hi - 8))), -8, 7) + 8.
+ * The draft W4 = (hi - 8) s is then within s/2 of W and the target W8 within
+ * s/16 (s/32 where lo is not clamped).
+ *   w      : fp16 [N, K] weights (finite).
+ *   hi, lo : uint8 [N, K/2] planes (outputs, the card's byte layout).
+ *   scale  : fp16 [N, K/128] (output).
+ * K must be a positive multiple of 128; checks and errors as the other
+ * entry points.
+ */
+int bitnest_pack_weights(const uint16_t *w, int64_t N, int64_t K, uint8_t *hi, uint8_t *lo,
+                         uint16_t *scale, void *stream);
+
+/*
  * Pack unpacked nibbles into the planes of the model card's layout
  * ("Files": byte j holds column 2j in its low nibble, 2j+1 in its high).
  *   uh, ul : uint8 [N, K] nibble values; only the low 4 bits are used.

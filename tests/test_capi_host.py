@@ -165,3 +165,12 @@ def test_linear_ws_argument_checks(L):
     assert call(K=200) == 2
     assert call(path=7) == 1
     assert call(M=0) == 0
+
+
+def test_pack_weights_argument_checks(L):
+    v = ctypes.c_void_p
+    assert L.bitnest_pack_weights(v(A), 4, 200, v(A), v(A), v(A), None) == 2
+    assert L.bitnest_pack_weights(None, 4, 128, v(A), v(A), v(A), None) == 1
+    assert L.bitnest_pack_weights(v(A), 4, 128, v(A), None, v(A), None) == 1
+    assert L.bitnest_pack_weights(v(A), 4, 128, v(A), v(A), v(MIS), None) == 3
+    assert L.bitnest_pack_weights(v(A), 0, 128, None, None, None, None) == 0

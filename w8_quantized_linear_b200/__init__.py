@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
     L.bitnest_device_wait_timeout.argtypes = [I]
     L.bitnest_device_wait_timeout.restype = I
     L.bitnest_pack_planes.argtypes = [P, P, I64, I64, P, P, P]
+    L.bitnest_pack_weights.argtypes = [P, I64, I64, P, P, P, P]
     L.bitnest_quantize_act.argtypes = [P, I64, I64, I, P, P, P, P]
     L.bitnest_act_group_sums.argtypes = [P, I64, I64, P, P]
     L.bitnest_linear.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, P]
@@ -64,7 +65,8 @@ def lib() -> ctypes.CDLL:
     L.bitnest_linear_static_ws.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, I, P]
     L.bitnest_linear_ws_bytes.argtypes = [I, I64, I64, I64, I]
     L.bitnest_linear_ws_bytes.restype = I64
-    for name in ("bitnest_pack_planes", "bitnest_quantize_act", "bitnest_act_group_sums",
+    for name in ("bitnest_pack_planes", "bitnest_pack_weights", "bitnest_quantize_act",
+                 "bitnest_act_group_sums",
                  "bitnest_linear", "bitnest_linear_path", "bitnest_select_path",
                  "bitnest_debug_group_sums", "bitnest_quantize_linear", "bitnest_linear_ws",
                  "bitnest_linear_static_ws"):
@@ -115,6 +117,22 @@ def pack_planes(uh, ul=None):
     _check(lib().bitnest_pack_planes(_ptr(uh), _ptr(ul), N, K, _ptr(hi), _ptr(lo), _stream(uh)),
            "bitnest_pack_planes")
     return hi, lo
+
+
+def pack_weights(w, out=None):
+    """fp16 weights [N, K] -> (hi, lo uint8 [N, K/2], scale fp16 [N, K/128]):
+    round-to-nearest 4-bit high nibble, closed-form residual low nibble."""
+    import torch
+
+    N, K = w.shape
+    if out is None:
+        out = (torch.empty((N, K // 2), dtype=torch.uint8, device=w.device),
+               torch.empty((N, K // 2), dtype=torch.uint8, device=w.device),
+               torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device))
+    hi, lo, sc = out
+    _check(lib().bitnest_pack_weights(_ptr(w), N, K, _ptr(hi), _ptr(lo), _ptr(sc), _stream(w)),
+           "bitnest_pack_weights")
+    return hi, lo, sc
 
 
 def quantize_act(x, act_group: int = 0, with_sum: bool = True, out=None):

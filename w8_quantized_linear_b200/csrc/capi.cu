@@ -102,6 +102,17 @@ int bitnest_pack_planes(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t
   return cuda_status(launch_pack(uh, ul, N, K, hi, lo, (cudaStream_t)stream));
 }
 
+int bitnest_pack_weights(const uint16_t *w, int64_t N, int64_t K, uint8_t *hi, uint8_t *lo,
+                         uint16_t *scale, void *stream) {
+  int s = check_shape(0, N, K);
+  if (s != BITNEST_OK) return s;
+  if (N == 0) return BITNEST_OK;
+  if (!w || !hi || !lo || !scale) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(w) || misaligned(hi) || misaligned(lo) || misaligned(scale))
+    return BITNEST_ERR_MISALIGNED;
+  return cuda_status(launch_pack_weights(w, N, K, hi, lo, scale, (cudaStream_t)stream));
+}
+
 int bitnest_quantize_act(const uint16_t *x, int64_t M, int64_t K, int act_group, int8_t *xq,
                          float *xscale, int32_t *xsum, void *stream) {
   if (act_group != 0 && act_group != kGroup) return BITNEST_ERR_INVALID_ARG;

@@ -28,6 +28,8 @@ struct LinearArgs {
 
 cudaError_t launch_pack(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K, uint8_t *hi,
                         uint8_t *lo, cudaStream_t st);
+cudaError_t launch_pack_weights(const uint16_t *w, int64_t N, int64_t K, uint8_t *hi,
+                                uint8_t *lo, uint16_t *scale, cudaStream_t st);
 cudaError_t launch_quantize(const uint16_t *x, int64_t M, int64_t K, int act_group, int8_t *xq,
                             float *xs, int32_t *xsum, cudaStream_t st);
 cudaError_t launch_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,

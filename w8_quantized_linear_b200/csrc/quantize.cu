@@ -32,6 +32,69 @@ cudaError_t launch_pack(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t
   return cudaGetLastError();
 }
 
+// --------------------------------------------------- packer from weights
+// BitNest-Llama-3-8B model card, opening paragraph (the high nibble a 4-bit
+// model fitted first, the low nibble the closed-form residual back to 8
+// bits) and section "Files" (u = q + 8, fp16 scale per 128 columns).  The
+// card fits the high nibble by GPTQ; here it is rounded to nearest:
+//   s = fp16(max|W| / 7) per row and group, t = W / s (fp32, correctly
+//   rounded), q4 = rne(t) (|t| <= 7.007: no clamp needed),
+//   ql = clamp(rne(16 (t - q4)), -8, 7), planes u = q + 8; s = 0 for an
+//   all-zero group (both nibbles 8).
+// One warp per (row, group): lane i holds columns 4i .. 4i+3.
+__global__ void __launch_bounds__(256) pack_weights_kernel(const uint16_t *__restrict__ w,
+                                                           int64_t N, int64_t K,
+                                                           uint8_t *__restrict__ hi,
+                                                           uint8_t *__restrict__ lo,
+                                                           uint16_t *__restrict__ scale) {
+  const int64_t G = K / kGroup;
+  const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= N * G) return;  // whole warps leave together
+  const int64_t n = wid / G, g = wid - n * G;
+  const int64_t k0 = g * kGroup + 4 * lane;
+  const uint2 raw = *reinterpret_cast<const uint2 *>(w + n * K + k0);
+  const __half2 h01 = *reinterpret_cast<const __half2 *>(&raw.x);
+  const __half2 h23 = *reinterpret_cast<const __half2 *>(&raw.y);
+  const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+  const float v[4] = {f01.x, f01.y, f23.x, f23.y};
+  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const __half sh = __float2half_rn(__fdiv_rn(amax, 7.0f));
+  const float sf = __half2float(sh);
+  uint32_t uh[4], ul[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int q4 = 0, ql = 0;
+    if (sf != 0.0f) {
+      const float t = __fdiv_rn(v[i], sf);
+      const float r4 = rintf(t);  // round half to even
+      q4 = (int)r4;
+      ql = __float2int_rn(__fmul_rn(16.0f, __fsub_rn(t, r4)));
+      ql = max(-8, min(7, ql));
+    }
+    uh[i] = (uint32_t)(q4 + 8);
+    ul[i] = (uint32_t)(ql + 8);
+  }
+  // plane bytes j = k / 2: column 2j in the low nibble, 2j+1 in the high one
+  const uint16_t hb = (uint16_t)((uh[0] | (uh[1] << 4)) | ((uh[2] | (uh[3] << 4)) << 8));
+  const uint16_t lb = (uint16_t)((ul[0] | (ul[1] << 4)) | ((ul[2] | (ul[3] << 4)) << 8));
+  *reinterpret_cast<uint16_t *>(hi + n * (K / 2) + k0 / 2) = hb;
+  *reinterpret_cast<uint16_t *>(lo + n * (K / 2) + k0 / 2) = lb;
+  if (lane == 0) scale[n * G + g] = __half_as_ushort(sh);
+}
+
+cudaError_t launch_pack_weights(const uint16_t *w, int64_t N, int64_t K, uint8_t *hi,
+                                uint8_t *lo, uint16_t *scale, cudaStream_t st) {
+  const int64_t warps = N * (K / kGroup);
+  const int threads = 256;
+  const int64_t blocks = (warps * 32 + threads - 1) / threads;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  pack_weights_kernel<<<(unsigned)blocks, threads, 0, st>>>(w, N, K, hi, lo, scale);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------ quantiser
 // One block per token.  Vector v (8 columns) is handled by thread v % T; a
 // group (16 vectors) is 16 consecutive threads of one pass.  With V > 0 every
