@@ -62,6 +62,12 @@ def _load():
     lib.oracle_float_to_half.argtypes = [ctypes.c_float]
     lib.oracle_float_to_half.restype = ctypes.c_uint16
     lib.oracle_pack_weights.argtypes = [P, I64, I64, P, P, P]
+    lib.oracle_h28.argtypes = [I, I]
+    lib.oracle_h28.restype = I
+    lib.oracle_hadamard_entry.argtypes = [I64, I64, I64]
+    lib.oracle_hadamard_entry.restype = I
+    lib.oracle_hadamard_rotate.argtypes = [P, I64, I64, P]
+    lib.oracle_quantize_f32.argtypes = [P, I64, I64, P, P]
     lib.oracle_pack_plane.argtypes = [P, I64, I64, P]
     lib.oracle_unpack_plane.argtypes = [P, I64, I64, P]
     lib.oracle_dequant.argtypes = [I, P, P, P, I64, I64, P]
@@ -119,6 +125,46 @@ def pack_weights(w):
     sc = np.empty((N, K // GROUP), np.uint16)
     _load().oracle_pack_weights(_ptr(wb), N, K, _ptr(uh), _ptr(ul), _ptr(sc))
     return uh, ul, sc
+
+
+def h28() -> np.ndarray:
+    """The order-28 Hadamard factor (Paley construction I over GF(27))."""
+    lib = _load()
+    return np.array([[lib.oracle_h28(i, j) for j in range(28)] for i in range(28)], np.int64)
+
+
+def hadamard_matrix(K: int) -> np.ndarray:
+    """H [K, K] (+-1) of the rotation; small K only (entry by entry)."""
+    lib = _load()
+    return np.array([[lib.oracle_hadamard_entry(K, i, j) for j in range(K)] for i in range(K)],
+                    np.int64)
+
+
+def hadamard_rotate(x) -> np.ndarray:
+    """fp16 [M, K] -> fp64 x H / sqrt(K) (K a power of two or 28 times one)."""
+    xb = _half_bits(x)
+    M, K = xb.shape
+    out = np.empty((M, K), np.float64)
+    _load().oracle_hadamard_rotate(_ptr(xb), M, K, _ptr(out))
+    return out
+
+
+def quantize_f32(x):
+    """fp32 [M, K] -> (q int8 [M, K], xs fp32 [M]): the per-token quantiser."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    q = np.empty((M, K), np.int8)
+    xs = np.empty((M,), np.float32)
+    _load().oracle_quantize_f32(_ptr(x), M, K, _ptr(q), _ptr(xs))
+    return q, xs
+
+
+def hadamard_quantize(x):
+    """The down_proj input path: rotate (fp64), round to fp32, quantise per
+    token.  Returns (q, xs, x_rot fp64)."""
+    xr = hadamard_rotate(x)
+    q, xs = quantize_f32(xr.astype(np.float32))
+    return q, xs, xr
 
 
 def pack_plane(u: np.ndarray) -> np.ndarray:

@@ -193,6 +193,103 @@ void oracle_pack_weights(const uint16_t *w, int64_t N, int64_t K, uint8_t *uh, u
     }
 }
 
+/* ---- online Hadamard rotation of the down_proj input ---------------------
+ * Model card, model table row "Rotation": an online Hadamard (R4) on the
+ * down_proj inputs; the card ships the matrices, not their construction.
+ * Reading: x_rot = x H / sqrt(K) with H a Hadamard matrix of order K:
+ *   K = 2^b       : Sylvester's matrix, H[i][j] = (-1)^popcount(i & j);
+ *   K = 28 * 2^b  : H = H28 (x) H_{2^b} (Kronecker product, the order-28
+ *                   factor outer: index i = i28 * 2^b + i'), H28 = I + S from
+ *                   Paley's construction I over GF(27): S = [[0, 1^T],
+ *                   [-1, Q]], Q[a][b] = chi(a - b), chi the quadratic
+ *                   character of GF(27) = GF(3)[x] / (x^3 - x - 1).
+ * Computed from the definition, one output at a time in fp64.          */
+static int gf27_add(int a, int b) {
+  int r = 0, p = 1;
+  for (int d = 0; d < 3; ++d, a /= 3, b /= 3, p *= 3) r += ((a % 3 + b % 3) % 3) * p;
+  return r;
+}
+static int gf27_neg(int a) {
+  int r = 0, p = 1;
+  for (int d = 0; d < 3; ++d, a /= 3, p *= 3) r += ((3 - a % 3) % 3) * p;
+  return r;
+}
+static int gf27_mul(int a, int b) {
+  /* polynomial product of a0 + a1 x + a2 x^2 and b0 + b1 x + b2 x^2, reduced
+   * with x^3 = x + 1 and x^4 = x^2 + x */
+  int ac[3] = {a % 3, a / 3 % 3, a / 9}, bc[3] = {b % 3, b / 3 % 3, b / 9};
+  int c[5] = {0, 0, 0, 0, 0};
+  for (int i = 0; i < 3; ++i)
+    for (int j = 0; j < 3; ++j) c[i + j] += ac[i] * bc[j];
+  c[1] += c[3]; c[0] += c[3]; /* x^3 -> x + 1 */
+  c[2] += c[4]; c[1] += c[4]; /* x^4 -> x^2 + x */
+  return c[0] % 3 + 3 * (c[1] % 3) + 9 * (c[2] % 3);
+}
+/* H28[i][j] in {+1, -1} */
+int oracle_h28(int i, int j) {
+  static int chi[27];
+  static int ready = 0;
+  if (!ready) {
+    for (int a = 0; a < 27; ++a) chi[a] = -1;
+    chi[0] = 0;
+    for (int a = 1; a < 27; ++a) chi[gf27_mul(a, a)] = 1;
+    ready = 1;
+  }
+  int sij;
+  if (i == j) return 1; /* H = I + S, S has a zero diagonal */
+  if (i == 0) sij = 1;
+  else if (j == 0) sij = -1;
+  else sij = chi[gf27_add(i - 1, gf27_neg(j - 1))];
+  return sij;
+}
+static int popcount64(uint64_t v) {
+  int c = 0;
+  for (; v; v &= v - 1) ++c;
+  return c;
+}
+/* H[i][j] of order K (K a power of two, or 28 times one) */
+int oracle_hadamard_entry(int64_t K, int64_t i, int64_t j) {
+  int64_t p = (K % 28 == 0) ? K / 28 : K;
+  int s = (popcount64((uint64_t)((i % p) & (j % p))) & 1) ? -1 : 1;
+  if (K % 28 == 0) s *= oracle_h28((int)(i / p), (int)(j / p));
+  return s;
+}
+/* x fp16 [M, K] -> xr fp64 [M, K] = x H / sqrt(K) */
+void oracle_hadamard_rotate(const uint16_t *x, int64_t M, int64_t K, double *xr) {
+  double norm = 1.0 / sqrt((double)K);
+#pragma omp parallel for schedule(static)
+  for (int64_t j = 0; j < K; ++j)
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int64_t i = 0; i < K; ++i)
+        acc += oracle_half_to_double(x[m * K + i]) * (double)oracle_hadamard_entry(K, i, j);
+      xr[m * K + j] = acc * norm;
+    }
+}
+
+/* The activation quantiser on fp32 inputs (the rotated activations rounded
+ * to fp32): the same steps as oracle_quantize, per token.               */
+void oracle_quantize_f32(const float *x, int64_t M, int64_t K, int8_t *q, float *xs) {
+  for (int64_t m = 0; m < M; ++m) {
+    const float *xr = x + m * K;
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k)
+      if (fabsf(xr[k]) > amax) amax = fabsf(xr[k]);
+    float s = amax / 127.0f;
+    xs[m] = s;
+    for (int64_t k = 0; k < K; ++k) {
+      if (s == 0.0f) {
+        q[m * K + k] = 0;
+        continue;
+      }
+      float r = nearbyintf(xr[k] / s);
+      if (r > 127.0f) r = 127.0f;
+      if (r < -127.0f) r = -127.0f;
+      q[m * K + k] = (int8_t)r;
+    }
+  }
+}
+
 /* ---- symmetric int8 activation quantiser --------------------------------
  * Model card, model table row "Activations": symmetric int8 per token, and
  * per 128-column group for o_proj.  Readings where the card is silent:

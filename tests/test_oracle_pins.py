@@ -423,3 +423,69 @@ def test_pack_weights_error_bounds(oracle_mod):
     unclipped = ul < 15
     assert np.all(d8[unclipped] <= s[unclipped] / 32 * (1 + 2.0 ** -20))
     assert sc[1, 0] == 0 and np.all(uh[1, :128] == 8) and np.all(ul[1, :128] == 8)
+
+
+# ------------------------------------------------- Hadamard rotation (R4)
+def test_h28_is_a_skew_hadamard_matrix(oracle_mod):
+    """Paley construction I: entries +-1, H H^T = 28 I, and H - I skew-symmetric."""
+    H = oracle_mod.h28()
+    assert set(np.unique(H).tolist()) == {-1, 1}
+    assert np.array_equal(H @ H.T, 28 * np.eye(28, dtype=np.int64))
+    S = H - np.eye(28, dtype=np.int64)
+    assert np.array_equal(S.T, -S)
+
+
+@pytest.mark.parametrize("b", range(1, 8))
+def test_sylvester_factor_matches_scipy(oracle_mod, b):
+    scipy_linalg = pytest.importorskip("scipy.linalg")
+    assert np.array_equal(oracle_mod.hadamard_matrix(2 ** b), scipy_linalg.hadamard(2 ** b))
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_order_28_p_is_the_kronecker_product(oracle_mod, p):
+    """Index i = i28 * p + i': the order-28 factor outer (numpy's kron)."""
+    scipy_linalg = pytest.importorskip("scipy.linalg")
+    H = oracle_mod.hadamard_matrix(28 * p)
+    assert np.array_equal(H, np.kron(oracle_mod.h28(), scipy_linalg.hadamard(p)))
+    assert np.array_equal(H @ H.T, 28 * p * np.eye(28 * p, dtype=np.int64))
+
+
+@pytest.mark.parametrize("K", [128, 112, 224])
+def test_rotation_is_x_times_h_over_sqrt_k(oracle_mod, K):
+    """Small K: the oracle's rotation against numpy's fp64 matmul with H."""
+    x = synth.activations(4242 + K, 3, K)
+    H = oracle_mod.hadamard_matrix(K).astype(np.float64)
+    ref = x.astype(np.float64) @ H / np.sqrt(K)
+    assert np.allclose(oracle_mod.hadamard_rotate(x), ref, rtol=1e-13, atol=1e-13)
+
+
+def test_rotation_preserves_the_norm_at_down_proj_size(oracle_mod):
+    """K = 14336 = 28 * 512: orthogonal (Parseval), and a one-hot input gives
+    a row of H / sqrt(K)."""
+    K = 14336
+    x = synth.activations(4343, 1, K)
+    xr = oracle_mod.hadamard_rotate(x)
+    n0 = np.sum(x.astype(np.float64) ** 2)
+    assert abs(np.sum(xr ** 2) - n0) <= 1e-10 * n0
+    e = np.zeros((1, K), np.float16)
+    e[0, 1000] = 1.0
+    row = oracle_mod.hadamard_rotate(e)[0] * np.sqrt(K)
+    i28, ip = divmod(1000, 512)
+    scipy_linalg = pytest.importorskip("scipy.linalg")
+    ref = np.kron(oracle_mod.h28()[i28], scipy_linalg.hadamard(512)[ip])
+    assert np.allclose(row, ref, atol=1e-12)
+
+
+def test_quantize_f32_matches_numpy_and_fp16_path(oracle_mod):
+    """fp32 quantiser: numpy fp32 division and round-half-even; on fp16
+    values it equals the fp16 quantiser."""
+    x16 = synth.activations(4444, 5, 1024)
+    q, xs = oracle_mod.quantize_f32(x16.astype(np.float32))
+    q16, xs16 = oracle_mod.quantize(x16, 0)
+    assert np.array_equal(q, q16) and np.array_equal(xs, xs16)
+    x = (np.random.default_rng(5).standard_normal((4, 777)) * 3).astype(np.float32)
+    amax = np.max(np.abs(x), axis=1)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    ref = np.clip(np.rint(x / s[:, None]), -127, 127).astype(np.int8)
+    q, xs = oracle_mod.quantize_f32(x)
+    assert np.array_equal(xs, s) and np.array_equal(q, ref)
