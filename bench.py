@@ -584,6 +584,41 @@ def measure_sweep(wl, hbm_peak, reps=5):
     return res
 
 
+# ------------------------------------------- down_proj input: R4 rotation
+def measure_hadamard(wl, hbm_peak, reps=20):
+    """bitnest_hadamard_quantize_act (x H / sqrt(K) + per-token int8) on the
+    down_proj input (K = 14336) next to the plain quantiser, at the decode
+    batches and the prefill batch; one launch after a spin, CUDA events."""
+    import torch
+
+    bn = wl.bn
+    N, K, _ = synth.LLAMA3_8B_PROJECTIONS["down_proj"]
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    res = {}
+    for M in (1, 4, PREFILL_M):
+        x = torch.from_numpy(synth.activations(synth.SEED_ACTS + 500 + M, M, K)).to(wl.dev)
+        nbytes = 2 * M * K + M * K + 4 * M + 4 * M * (K // 128)
+        for name, fn in (("rotate+quantise", lambda: bn.hadamard_quantize_act(x)),
+                         ("quantise", lambda: bn.quantize_act(x, 0))):
+            fn()
+            t = 0.0
+            for _ in range(reps):
+                torch.cuda._sleep(200_000)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                t += a.elapsed_time(b) / 1e3
+            t /= reps
+            res[f"{name}/M={M}"] = {"us": round(t * 1e6, 2), "GB/s": round(nbytes / t / 1e9, 1),
+                                    "frac_hbm": round(nbytes / t / 1e9 / hbm_peak, 3)}
+        del x
+    return {"workload": "down_proj input (K = 14336 = 28 x 512): online Hadamard rotation "
+                        "fused with per-token int8 quantisation, vs the quantiser alone",
+            "per_case": res}
+
+
 # ------------------------------------------------ packer from fp weights
 def measure_pack(wl, hbm_peak, reps=5):
     """bitnest_pack_weights on the seven projections' shapes (seeded
@@ -712,7 +747,7 @@ def main():
                     help="launch the step's kernels directly instead of replaying a CUDA graph "
                          "(for profilers that cannot replay the captured kernel nodes)")
     ap.add_argument("--workload", default="all",
-                    choices=["all", "decode", "prefill", "sweep", "round", "pack"],
+                    choices=["all", "decode", "prefill", "sweep", "round", "pack", "hadamard"],
                     help="all: the decode step line with the prefill, M-sweep and "
                          "decode-round objects; otherwise only that part (profiling runs)")
     args = ap.parse_args()
@@ -756,6 +791,9 @@ def main():
     pack = None
     if args.workload in ("all", "pack"):
         pack = measure_pack(wl, hbm_peak)
+    had = None
+    if args.workload in ("all", "hadamard"):
+        had = measure_hadamard(wl, hbm_peak)
     prefill = None
     if args.workload in ("all", "prefill"):
         pre, pre_ops, pre_t = measure_prefill(wl, reps=10 if args.workload == "all" else 3)
@@ -777,7 +815,7 @@ def main():
             dist.destroy_process_group()
         if rank == 0:
             part = {"prefill": prefill, "m_sweep": sweep, "decode_round": rnd,
-                    "pack_from_weights": pack}
+                    "pack_from_weights": pack, "down_proj_input_rotation": had}
             print(json.dumps({"metric": METRIC, "workload": f"{args.workload} only",
                               **{k: v for k, v in part.items() if v is not None}}), flush=True)
         return
@@ -816,6 +854,8 @@ def main():
         out["decode_round"] = rnd
     if pack is not None:
         out["pack_from_weights"] = pack
+    if had is not None:
+        out["down_proj_input_rotation"] = had
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, cores, rows = cpu_baseline()
         out["cpu_baseline"] = {

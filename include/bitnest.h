@@ -109,6 +109,31 @@ int bitnest_pack_weights(const uint16_t *w, int64_t N, int64_t K, uint8_t *hi, u
                          uint16_t *scale, void *stream);
 
 /*
+ * The down_proj input path: online Hadamard rotation (model card, model
+ * table row "Rotation": R4 online Hadamard on down_proj inputs) fused with
+ * the per-token quantiser.  The card ships its R4 matrices, not their
+ * construction; this library's reading:
+ *   x_rot = x H / sqrt(K), H of order K:
+ *     K = p (a power of two)      : Sylvester's matrix (-1)^popcount(i & j);
+ *     K = 28 p (p a power of two) : H = H28 (x) H_p (Kronecker product, the
+ *        order-28 factor outer), H28 = I + S from Paley's construction I
+ *        over GF(27) = GF(3)[x] / (x^3 - x - 1).
+ *   Then, per token, as bitnest_quantize_act with act_group 0 on the fp32
+ *   rotated values: xscale = max|x_rot| / 127, xq = rne(x_rot / xscale),
+ *   xsum = per-128-group sums of xq.
+ * The rotation runs in fp32 (a Walsh-Hadamard transform per length-p block,
+ * then the order-28 mix), so x_rot carries fp32 rounding: a code may differ
+ * by one from that of the exact rotation where x_rot / xscale is within
+ * rounding of a half-integer.
+ *   x : fp16 [M, K];  xq : int8 [M, K];  xscale : fp32 [M];
+ *   xsum : int32 [M, K/128] or NULL.
+ * K must be p or 28 p as above, a multiple of 128 and at most 32768
+ * (else BITNEST_ERR_UNSUPPORTED_SHAPE); e.g. down_proj's K = 14336 = 28 x 512.
+ */
+int bitnest_hadamard_quantize_act(const uint16_t *x, int64_t M, int64_t K, int8_t *xq,
+                                  float *xscale, int32_t *xsum, void *stream);
+
+/*
  * Pack unpacked nibbles into the planes of the model card's layout
  * ("Files": byte j holds column 2j in its low nibble, 2j+1 in its high).
  *   uh, ul : uint8 [N, K] nibble values; only the low 4 bits are used.

@@ -174,3 +174,13 @@ def test_pack_weights_argument_checks(L):
     assert L.bitnest_pack_weights(v(A), 4, 128, v(A), None, v(A), None) == 1
     assert L.bitnest_pack_weights(v(A), 4, 128, v(A), v(A), v(MIS), None) == 3
     assert L.bitnest_pack_weights(v(A), 0, 128, None, None, None, None) == 0
+
+
+def test_hadamard_quantize_argument_checks(L):
+    v = ctypes.c_void_p
+    assert L.bitnest_hadamard_quantize_act(v(A), 2, 1000, v(A), v(A), None, None) == 2
+    assert L.bitnest_hadamard_quantize_act(v(A), 2, 384, v(A), v(A), None, None) == 2  # not p, 28p
+    assert L.bitnest_hadamard_quantize_act(v(A), 2, 65536, v(A), v(A), None, None) == 2  # too long
+    assert L.bitnest_hadamard_quantize_act(None, 2, 14336, v(A), v(A), None, None) == 1
+    assert L.bitnest_hadamard_quantize_act(v(A), 2, 14336, v(MIS), v(A), None, None) == 3
+    assert L.bitnest_hadamard_quantize_act(v(A), 0, 14336, None, None, None, None) == 0

@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
     L.bitnest_device_wait_timeout.restype = I
     L.bitnest_pack_planes.argtypes = [P, P, I64, I64, P, P, P]
     L.bitnest_pack_weights.argtypes = [P, I64, I64, P, P, P, P]
+    L.bitnest_hadamard_quantize_act.argtypes = [P, I64, I64, P, P, P, P]
     L.bitnest_quantize_act.argtypes = [P, I64, I64, I, P, P, P, P]
     L.bitnest_act_group_sums.argtypes = [P, I64, I64, P, P]
     L.bitnest_linear.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, P]
@@ -66,7 +67,7 @@ def lib() -> ctypes.CDLL:
     L.bitnest_linear_ws_bytes.argtypes = [I, I64, I64, I64, I]
     L.bitnest_linear_ws_bytes.restype = I64
     for name in ("bitnest_pack_planes", "bitnest_pack_weights", "bitnest_quantize_act",
-                 "bitnest_act_group_sums",
+                 "bitnest_act_group_sums", "bitnest_hadamard_quantize_act",
                  "bitnest_linear", "bitnest_linear_path", "bitnest_select_path",
                  "bitnest_debug_group_sums", "bitnest_quantize_linear", "bitnest_linear_ws",
                  "bitnest_linear_static_ws"):
@@ -149,6 +150,22 @@ def quantize_act(x, act_group: int = 0, with_sum: bool = True, out=None):
         xq, xs, xsum = out
     _check(lib().bitnest_quantize_act(_ptr(x), M, K, int(act_group), _ptr(xq), _ptr(xs),
                                       _ptr(xsum), _stream(x)), "bitnest_quantize_act")
+    return xq, xs, xsum
+
+
+def hadamard_quantize_act(x, out=None):
+    """down_proj input path: fp16 [M, K] -> rotated by x H / sqrt(K) and
+    quantised per token: (xq int8 [M, K], xscale fp32 [M], xsum int32 [M, K/128])."""
+    import torch
+
+    M, K = x.shape
+    if out is None:
+        out = (torch.empty((M, K), dtype=torch.int8, device=x.device),
+               torch.empty((M,), dtype=torch.float32, device=x.device),
+               torch.empty((M, K // GROUP), dtype=torch.int32, device=x.device))
+    xq, xs, xsum = out
+    _check(lib().bitnest_hadamard_quantize_act(_ptr(x), M, K, _ptr(xq), _ptr(xs), _ptr(xsum),
+                                               _stream(x)), "bitnest_hadamard_quantize_act")
     return xq, xs, xsum
 
 

@@ -126,6 +126,18 @@ int bitnest_quantize_act(const uint16_t *x, int64_t M, int64_t K, int act_group,
   return cuda_status(launch_quantize(x, M, K, act_group, xq, xscale, xsum, (cudaStream_t)stream));
 }
 
+int bitnest_hadamard_quantize_act(const uint16_t *x, int64_t M, int64_t K, int8_t *xq,
+                                  float *xscale, int32_t *xsum, void *stream) {
+  int s = check_shape(M, 0, K);
+  if (s != BITNEST_OK) return s;
+  if (!hadamard_supported(K)) return BITNEST_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return BITNEST_OK;
+  if (!x || !xq || !xscale) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(x) || misaligned(xq) || misaligned(xscale) || (xsum && misaligned(xsum)))
+    return BITNEST_ERR_MISALIGNED;
+  return cuda_status(launch_hadamard_quantize(x, M, K, xq, xscale, xsum, (cudaStream_t)stream));
+}
+
 int bitnest_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
                            void *stream) {
   int s = check_shape(M, 0, K);

@@ -34,6 +34,11 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t M, int64_t K, int act_gro
                             float *xs, int32_t *xsum, cudaStream_t st);
 cudaError_t launch_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
                                   cudaStream_t st);
+// Hadamard rotation x H / sqrt(K) + per-token quantisation (K = p or 28 p,
+// p a power of two, K <= 32768).
+bool hadamard_supported(int64_t K);
+cudaError_t launch_hadamard_quantize(const uint16_t *x, int64_t M, int64_t K, int8_t *xq,
+                                     float *xs, int32_t *xsum, cudaStream_t st);
 
 // Largest M * K the GEMV kernels can stage in shared memory.
 bool gemv_fits(int64_t M, int64_t K);
