@@ -80,15 +80,15 @@ struct Params {
 struct TileCoord {
   int tmn, split, n0, m0, g0, g1;
 };
-template <int BT>
+template <int BT, bool SPLIT>
 __device__ __forceinline__ TileCoord tile_coord(const Params &p, int tile) {
   TileCoord c;
-  c.split = tile % p.splits;
-  c.tmn = tile / p.splits;
+  c.split = SPLIT ? tile % p.splits : 0;
+  c.tmn = SPLIT ? tile / p.splits : tile;
   c.n0 = (c.tmn / p.mt) * BW;
   c.m0 = (c.tmn % p.mt) * BT;
-  c.g0 = c.split * p.gps;
-  c.g1 = min(p.G, c.g0 + p.gps);
+  c.g0 = SPLIT ? c.split * p.gps : 0;
+  c.g1 = SPLIT ? min(p.G, c.g0 + p.gps) : p.G;
   return c;
 }
 
@@ -132,7 +132,7 @@ __device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
-template <int MODE, int BT, bool ACTG, bool DEBUG>
+template <int MODE, int BT, bool ACTG, bool DEBUG, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_linear_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_hi,
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;  // stage slot and the parity of its current fill
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-      const TileCoord tc = tile_coord<BT>(p, tile);
+      const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
       for (int g = tc.g0; g < tc.g1; ++g) {
         ok = mbar_wait_warp(&fullB[s], ph);
         if (!ok) break;
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       constexpr uint32_t bytes = BT * 128 + BW * 64 * (MODE ? 2 : 1);
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-        const TileCoord tc = tile_coord<BT>(p, tile);
+        const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
         const int n0 = tc.n0, m0 = tc.m0;
         for (int g = tc.g0; g < tc.g1; ++g, ++it) {
           if (!mbar_wait(&stageFree[s], ph ^ 1u)) {
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint64_t kStageDesc = STAGE >> 4;  // descriptor address unit: 16 bytes
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-        const TileCoord tc = tile_coord<BT>(p, tile);
+        const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
         for (int g = tc.g0; g < tc.g1; ++g, ++it) {
           ok = mbar_wait(&fullB[s], ph) && mbar_wait(&fullA[s], ph) &&
                mbar_wait(&accEmpty[b], bph ^ 1u);
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-      const TileCoord tc = tile_coord<BT>(p, tile);
+      const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
       const int n0 = tc.n0, m0 = tc.m0, G1 = tc.g1;
       for (int gb = tc.g0; gb < G1 && ok; gb += kCBatch) {
         uint16_t sv[4][kCBatch];
@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-      const TileCoord tc = tile_coord<BT>(p, tile);
+      const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
       const int n = tc.n0 + row, m0 = tc.m0;
       float acc[COLS];
 #pragma unroll
@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&emptyC[cs]);
         }
       }
-      if (!DEBUG && ok && p.splits > 1) {
+      if (SPLIT && !DEBUG && ok) {
         // this range's partial sums of the warp's sub-block (rows of its lane
         // quarter, its columns), then one arrival per warp; the last of the
         // splits to arrive adds them all in split order
@@ -591,6 +591,8 @@ SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int bt) {
 
 template <int MODE, int BT, bool ACTG, bool DEBUG>
 cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
+  // split K only where the plan asks for it: the unsplit kernel carries none
+  // of the partial-tile code
   const int G = (int)(a.K / kGroup);
   const int stages = pick_stages(MODE, BT, kMaxSmem);
   if (stages == 0) return cudaErrorInvalidValue;
@@ -637,7 +639,8 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   p.stages = stages;
   const int grid = p.tiles < num_sms() ? p.tiles : num_sms();
   const int smem = smem_total(MODE, BT, stages);
-  auto kern = tc_linear_kernel<MODE, BT, ACTG, DEBUG>;
+  auto kern = p.splits > 1 ? tc_linear_kernel<MODE, BT, ACTG, DEBUG, !DEBUG>
+                           : tc_linear_kernel<MODE, BT, ACTG, DEBUG, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, a.overlap, mq, mh,
