@@ -50,10 +50,11 @@ constexpr int kSegs = kStepCols / 256;                 // 128-byte plane segment
 constexpr int kPlaneBytes = kRows * kStepCols / 2;     // 32 KB: one TMA box per plane
 constexpr int kMaxStages = 8;
 constexpr int kRedSlots = 4;  // row blocks whose partial sums can be in flight
-// Weight stages the producer issues before the activations are loaded: the
-// stream starts while the preceding kernel runs, yet the memory queues are
-// short again when the consumers' activation loads go out.
-constexpr int kPreStages = 2;
+// Weight bytes the producer issues (per CTA) before the activations are
+// loaded: the stream starts while the preceding kernel runs, yet the memory
+// queues are short again when the consumers' activation loads go out (two
+// draft stages, one target stage).
+constexpr int kPreBytes = 64 * 1024;
 constexpr int kScaleSmemMax = 32 * 1024;  // the CTA's group scales are staged once
 constexpr int kSmemBudget = 227 * 1024;
 
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < p.nks; ++ks, ++it) {
           const int s = it % S;
           // the rest of the stream queues behind the activation loads
-          if (it == kPreStages && !mbar_wait(act_issued, 0)) {
+          if (it == kPreBytes / STAGE && !mbar_wait(act_issued, 0)) {
             ok = false;
             break;
           }
