@@ -205,7 +205,13 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t M, int64_t K, int act_gro
                             float *xs, int32_t *xsum, cudaStream_t st) {
   // programmatic dependent launch: the kernel waits for its predecessor first
   cudaError_t e;
-  if (act_group == 0) {
+  if (act_group == 0 && K / 8 > 2 * 256 && K / 8 <= 4 * 1024) {
+    // long rows (down_proj's K = 14336): 1024 threads, at most 4 vectors each
+    constexpr int T = 1024;
+    const int64_t per = (K / 8 + T - 1) / T;
+    auto kern = per <= 2 ? quantize_token_kernel<T, 2> : quantize_token_kernel<T, 4>;
+    e = launch_pdl(kern, dim3((unsigned)M), dim3(T), 0, st, true, x, K, xq, xs, xsum);
+  } else if (act_group == 0) {
     constexpr int T = 256;
     const int64_t per = (K / 8 + T - 1) / T;  // vectors per thread
     auto kern = per <= 1 ? quantize_token_kernel<T, 1>
