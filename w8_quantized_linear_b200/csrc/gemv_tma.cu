@@ -71,10 +71,11 @@ struct Params {
 
 __host__ __device__ constexpr int stage_bytes(int mode) { return (mode ? 2 : 1) * kPlaneBytes; }
 
-// row pitch (halves) of the staged group scales: an odd number of 8-byte
-// units, so rows stay 8-byte aligned and the 8 rows a warp reads with one
-// 8-byte load each fall in different banks
-__host__ __device__ inline int scale_pitch(int G) { return 4 * (((G + 3) / 4) | 1); }
+// row pitch (halves) of the staged group scales: an odd number of 16-byte
+// units, so rows are copied in 16-byte pieces and the 8 rows a warp reads
+// with one 8-byte load each fall in different banks (row r starts at bank
+// 4 (odd r mod 8))
+__host__ __device__ inline int scale_pitch(int G) { return 8 * (((G + 7) / 8) | 1); }
 
 // staged activations [M][2][Cp] x 16 B, group sums [Gp][8], group act. scales
 // [Gp][8], the CTA's group scales [nb * 16][pitch] fp16, partial-sum slots
@@ -119,9 +120,9 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, uint64_
 // loads of a warp hit 32 different banks.
 __device__ __forceinline__ int perm_row(int g) { return (g >> 1) + ((g & 1) << 2); }
 
-// Asynchronous 4-byte copy global -> shared.
-__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+// Asynchronous 16-byte copy global -> shared (L2 only).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() {
@@ -257,19 +258,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ------------------------------------------------------------- consumers
   constexpr int NT = kConsumerWarps * 32;
-  // The group scales of every row this CTA owns (32-bit words), copied
-  // asynchronously: all of them are in flight at once.  Like the planes they
-  // do not come from the preceding kernel, so this starts before the wait.
+  // The group scales of every row this CTA owns (16-byte pieces: G is a
+  // multiple of 8), copied asynchronously: all of them are in flight at
+  // once.  Like the planes they do not come from the preceding kernel, so
+  // this starts before the wait.
   if (!DEBUG) {
-    const int wpr = G / 2;  // G is even (a multiple of 8)
-    for (int i = threadIdx.x; i < nb * kRows * wpr; i += NT) {
-      const int rl = i / wpr, wd = i - rl * wpr;
+    const int cpr = G / 8;
+    for (int i = threadIdx.x; i < nb * kRows * cpr; i += NT) {
+      const int rl = i / cpr, c = i - rl * cpr;
       const int n = ((int)blockIdx.x + (rl / kRows) * (int)gridDim.x) * kRows + rl % kRows;
-      uint32_t *dst = reinterpret_cast<uint32_t *>(ssc + rl * sp) + wd;
+      uint4 *dst = reinterpret_cast<uint4 *>(ssc + rl * sp) + c;
       if (n < p.N)
-        cp_async4(dst, reinterpret_cast<const uint32_t *>(p.scale + (int64_t)n * G) + wd);
+        cp_async16(dst, reinterpret_cast<const uint4 *>(p.scale + (int64_t)n * G) + c);
       else
-        *dst = 0u;
+        *dst = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   griddep_wait();  // the activations are written by the preceding kernel
