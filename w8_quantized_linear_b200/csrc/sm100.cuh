@@ -1,5 +1,5 @@
 // sm_100a primitives in inline PTX: mbarriers with bounded waits, TMA tile
-// loads (no multicast), tcgen05 tensor memory, UMMA descriptors and MMA.
+// loads into this CTA only, tcgen05 tensor memory, UMMA descriptors and MMA.
 #pragma once
 
 #include <stdint.h>
@@ -67,7 +67,7 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity) {
 }
 
 // --------------------------------------------------------------------- TMA
-// 2D tile load global -> shared, completion counted on `bar` (no multicast).
+// 2D tile load global -> this CTA's shared memory, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, uint64_t *bar, int x,
                                             int y) {
   asm volatile(

@@ -25,7 +25,7 @@
 // Warp roles (15 warps):
 //   0..3   plane -> byte operand (shared-memory planes -> swizzled K-major)
 //   4      TMA producer: activation tile (128-byte swizzle) and the hi / lo
-//          plane tiles of the group, one mbarrier per stage (no multicast)
+//          plane tiles of the group, one mbarrier per stage (this CTA only)
 //   5      TMEM owner and MMA issuer (one thread)
 //   6      per-group constants: row scales, magic - offset * activation group
 //          sum per token (and the per-group activation scale for o_proj)
