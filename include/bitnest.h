@@ -86,6 +86,14 @@ int bitnest_version(void);
  * the flag after reading it. */
 int bitnest_device_wait_timeout(int reset);
 
+/* Test hook for the flag above: launches one warp that waits, with the
+ * kernels' bounded wait (cut to 4096 polls), on an mbarrier that nothing
+ * arrives at.  The wait gives up, sets the flag and the kernel returns;
+ * nothing faults or hangs.  Asynchronous on `stream`; clear the flag with
+ * bitnest_device_wait_timeout(1) afterwards, or later bounded waits give up
+ * at once. */
+int bitnest_debug_wait_probe(void *stream);
+
 /*
  * Build the planes and scales of one layer from its fp16 weights
  * (BitNest-Llama-3-8B model card, opening paragraph: the high nibble is a

@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
     L.bitnest_device_wait_timeout.argtypes = [I]
     L.bitnest_device_wait_timeout.restype = I
     L.bitnest_pack_planes.argtypes = [P, P, I64, I64, P, P, P]
+    L.bitnest_debug_wait_probe.argtypes = [P]
+    L.bitnest_debug_wait_probe.restype = I
     L.bitnest_pack_weights.argtypes = [P, I64, I64, P, P, P, P]
     L.bitnest_hadamard_quantize_act.argtypes = [P, I64, I64, P, P, P, P]
     L.bitnest_quantize_act.argtypes = [P, I64, I64, I, P, P, P, P]
@@ -102,6 +104,12 @@ def device_wait_timeout(reset: bool = False) -> int:
     if v < 0:
         raise BitnestError(-v, "bitnest_device_wait_timeout")
     return v
+
+
+def debug_wait_probe() -> None:
+    """Test hook: a kernel whose bounded wait gives up and sets the flag that
+    device_wait_timeout reports (clear it afterwards)."""
+    _check(lib().bitnest_debug_wait_probe(_stream()), "bitnest_debug_wait_probe")
 
 
 def select_path(mode: int, M: int, N: int, K: int) -> int:

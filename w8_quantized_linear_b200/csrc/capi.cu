@@ -90,6 +90,10 @@ int bitnest_device_wait_timeout(int reset) {
   return (f1 | f2) ? 1 : 0;
 }
 
+int bitnest_debug_wait_probe(void *stream) {
+  return cuda_status(launch_wait_probe((cudaStream_t)stream));
+}
+
 int bitnest_pack_planes(const uint8_t *uh, const uint8_t *ul, int64_t N, int64_t K,
                         uint8_t *hi, uint8_t *lo, void *stream) {
   int s = check_shape(0, N, K);

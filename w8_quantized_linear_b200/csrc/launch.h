@@ -61,5 +61,7 @@ cudaError_t tc_static_ws(void **ws);
 
 // The flag a bounded wait sets when it gives up (synchronous read).
 cudaError_t read_wait_timeout(int *flag, bool reset);
+// Test hook: a wait that gives up (sets the flag above).
+cudaError_t launch_wait_probe(cudaStream_t st);
 
 }  // namespace bitnest

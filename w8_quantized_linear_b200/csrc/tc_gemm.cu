@@ -670,6 +670,25 @@ cudaError_t launch_mode(const LinearArgs &a, cudaStream_t st) {
 
 }  // namespace tc
 
+// Test hook: one warp waits, with the kernels' own bounded wait (cut to 4096
+// polls), on an mbarrier that nothing ever arrives at.  The wait gives up
+// and sets this translation unit's g_wait_timeout, which read_wait_timeout
+// reports; nothing faults or hangs.
+__global__ void wait_probe_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  (void)mbar_wait(&bar, 0, 4096u);  // phase 0 never completes
+}
+
+cudaError_t launch_wait_probe(cudaStream_t st) {
+  wait_probe_kernel<<<1, 32, 0, st>>>();
+  return cudaGetLastError();
+}
+
 cudaError_t read_wait_timeout(int *flag, bool reset) {
   cudaError_t e = cudaMemcpyFromSymbol(flag, g_wait_timeout, sizeof(int));
   if (e != cudaSuccess || !reset) return e;
