@@ -264,3 +264,37 @@ def test_quantiser_near_ties_bit_exact(act_group):
             torch.cuda.synchronize()
             assert np.array_equal(host(fq), q)
             assert np.array_equal(host(fs), xs)
+
+
+# ---------------------------------- the bench's own launch configuration
+@pytest.mark.parametrize("members", [("gate_proj", "up_proj"), ("q_proj", "k_proj", "v_proj")],
+                         ids=["gate_up_N28672", "qkv_N6144"])
+def test_fused_layer_group_as_the_bench_launches_it(members):
+    """The decode step's fused weights (rows of the member projections
+    stacked: gate|up N = 28672, 13 row blocks per CTA; q|k|v N = 6144),
+    draft M=1 and target M=4 through the one-call entry with programmatic
+    dependent launch, as the bench times them; sampled rows against the
+    oracle, codes bit-exact."""
+    parts = [synth.LLAMA3_8B_PROJECTIONS[m] for m in members]
+    K, g = parts[0][1], parts[0][2]
+    uh = np.concatenate([synth.nibbles(synth.SEED_WEIGHTS + synth.PROJ_IDS[m], synth.STREAM_HI,
+                                       synth.LLAMA3_8B_PROJECTIONS[m][0], K) for m in members])
+    ul = np.concatenate([synth.nibbles(synth.SEED_WEIGHTS + synth.PROJ_IDS[m], synth.STREAM_LO,
+                                       synth.LLAMA3_8B_PROJECTIONS[m][0], K) for m in members])
+    s = np.concatenate([synth.group_scales(synth.SEED_SCALES + synth.PROJ_IDS[m],
+                                           synth.LLAMA3_8B_PROJECTIONS[m][0], K) for m in members])
+    N = uh.shape[0]
+    d_hi, d_lo = bn.pack_planes(dev(uh), dev(ul))
+    d_s = dev(s)
+    rows = _sample_rows(N, count=64, seed=N)
+    hi_r, lo_r = oracle.pack_plane(uh[rows]), oracle.pack_plane(ul[rows])
+    for mode, M in ((0, 1), (1, 4)):
+        x = synth.activations(synth.SEED_ACTS + N + mode, M, K)
+        y, (xq, xs, _) = bn.quantize_linear(mode, d_hi, d_lo, d_s, dev(x), g,
+                                            path=bn.PATH_AUTO | bn.PATH_OVERLAP)
+        torch.cuda.synchronize()
+        q, xs_ref = oracle.quantize(x, g)
+        assert np.array_equal(host(xq), q) and np.array_equal(host(xs), xs_ref)
+        y_ref = oracle.linear(mode, hi_r, lo_r if mode else None, s[rows], q, xs_ref, K, g)
+        assert oracle.max_normalised_error(host(y)[:, rows], y_ref) <= TOL
+    assert bn.device_wait_timeout(reset=True) == 0
