@@ -62,6 +62,7 @@ def _load():
     lib.oracle_float_to_half.argtypes = [ctypes.c_float]
     lib.oracle_float_to_half.restype = ctypes.c_uint16
     lib.oracle_pack_weights.argtypes = [P, I64, I64, P, P, P]
+    lib.oracle_nested_attention.argtypes = [I, P, I64, I64, I64, I64, P, P, P, P, P, P, P]
     lib.oracle_h28.argtypes = [I, I]
     lib.oracle_h28.restype = I
     lib.oracle_hadamard_entry.argtypes = [I64, I64, I64]
@@ -125,6 +126,29 @@ def pack_weights(w):
     sc = np.empty((N, K // GROUP), np.uint16)
     _load().oracle_pack_weights(_ptr(wb), N, K, _ptr(uh), _ptr(ul), _ptr(sc))
     return uh, ul, sc
+
+
+def kv_pack(kv):
+    """fp16 K or V rows [T * Hkv, D] -> (hi, lo planes [T * Hkv, D/2], fp16
+    scale bits [T * Hkv, D/128]): the runtime nesting of the cache (the
+    weights' packing rule, one group of 128 per row segment)."""
+    uh, ul, sc = pack_weights(kv)
+    return pack_plane(uh), pack_plane(ul), sc
+
+
+def nested_attention(mode: int, q, k_planes, v_planes, Hkv: int) -> np.ndarray:
+    """Decode attention of one token over a nested KV cache, fp64 [H, D].
+    q fp16 [H, D]; k_planes / v_planes = kv_pack(...) of [T * Hkv, D] rows
+    (row t * Hkv + j: token t, KV head j); draft reads hi, target hi and lo."""
+    qb = _half_bits(q)
+    H, D = qb.shape
+    k_hi, k_lo, k_sc = (_c(a, t) for a, t in zip(k_planes, (np.uint8, np.uint8, np.uint16)))
+    v_hi, v_lo, v_sc = (_c(a, t) for a, t in zip(v_planes, (np.uint8, np.uint8, np.uint16)))
+    T = k_hi.shape[0] // Hkv
+    out = np.empty((H, D), np.float64)
+    _load().oracle_nested_attention(mode, _ptr(qb), H, Hkv, D, T, _ptr(k_hi), _ptr(k_lo),
+                                    _ptr(k_sc), _ptr(v_hi), _ptr(v_lo), _ptr(v_sc), _ptr(out))
+    return out
 
 
 def h28() -> np.ndarray:

@@ -193,6 +193,60 @@ void oracle_pack_weights(const uint16_t *w, int64_t N, int64_t K, uint8_t *uh, u
     }
 }
 
+/* ---- nested KV cache: decode attention -----------------------------------
+ * Model card, model table row "KV cache": nested at runtime, the draft reads
+ * KV4, the target KV8.  The card gives no layout; the reading taken is the
+ * weights' nesting applied to the cache: every K (and V) row of one token and
+ * one KV head (head_dim = 128 values, one group) is packed at runtime with
+ * oracle_pack_weights' rule (fp16 scale max|x| / 7, round-to-nearest high
+ * nibble, closed-form residual low nibble); the draft dequantises
+ * (hi - 8) s, the target (16 (hi - 8) + (lo - 8)) s / 16.
+ * Decode attention of one new token, in fp64 from the definition:
+ *   head h (of H) reads KV head h / (H / Hkv)  (grouped-query attention);
+ *   score[t] = q_h . K[t] / sqrt(D), p = softmax(score) over t < T,
+ *   out_h = sum_t p[t] V[t].
+ * q: fp16 [H, D]; planes: uint8 [T * Hkv, D / 2] (row t * Hkv + j);
+ * scales: fp16 [T * Hkv, D / 128]; out: fp64 [H, D].                    */
+static double kv_value(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
+                       int64_t D, int64_t row, int64_t k) {
+  double s = oracle_half_to_double(scale[row * (D / ORACLE_GROUP) + k / ORACLE_GROUP]);
+  int h = nibble(hi, D, row, k);
+  if (mode == ORACLE_DRAFT) return (double)(h - 8) * s;
+  int l = nibble(lo, D, row, k);
+  return (double)(16 * (h - 8) + (l - 8)) * s / 16.0;
+}
+
+void oracle_nested_attention(int mode, const uint16_t *q, int64_t H, int64_t Hkv, int64_t D,
+                             int64_t T, const uint8_t *k_hi, const uint8_t *k_lo,
+                             const uint16_t *k_scale, const uint8_t *v_hi,
+                             const uint8_t *v_lo, const uint16_t *v_scale, double *out) {
+  double *score = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+  for (int64_t h = 0; h < H; ++h) {
+    int64_t j = h / (H / Hkv);
+    double mx = -INFINITY;
+    for (int64_t t = 0; t < T; ++t) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < D; ++k)
+        acc += oracle_half_to_double(q[h * D + k]) *
+               kv_value(mode, k_hi, k_lo, k_scale, D, t * Hkv + j, k);
+      score[t] = acc / sqrt((double)D);
+      if (score[t] > mx) mx = score[t];
+    }
+    double den = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+      score[t] = exp(score[t] - mx); /* shifted by the maximum: same softmax */
+      den += score[t];
+    }
+    for (int64_t k = 0; k < D; ++k) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < T; ++t)
+        acc += score[t] * kv_value(mode, v_hi, v_lo, v_scale, D, t * Hkv + j, k);
+      out[h * D + k] = acc / den;
+    }
+  }
+  free(score);
+}
+
 /* ---- online Hadamard rotation of the down_proj input ---------------------
  * Model card, model table row "Rotation": an online Hadamard (R4) on the
  * down_proj inputs; the card ships the matrices, not their construction.

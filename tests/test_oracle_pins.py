@@ -489,3 +489,63 @@ def test_quantize_f32_matches_numpy_and_fp16_path(oracle_mod):
     ref = np.clip(np.rint(x / s[:, None]), -127, 127).astype(np.int8)
     q, xs = oracle_mod.quantize_f32(x)
     assert np.array_equal(xs, s) and np.array_equal(q, ref)
+
+
+# ------------------------------------- nested KV cache: decode attention
+def _kv_case(seed, H, Hkv, D, T):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((H, D)).astype(np.float16)
+    k = (rng.standard_normal((T * Hkv, D)) * 0.7).astype(np.float16)
+    v = rng.standard_normal((T * Hkv, D)).astype(np.float16)
+    return q, k, v
+
+
+@pytest.mark.parametrize("H,Hkv,D,T", [(4, 2, 128, 7), (8, 8, 128, 3), (32, 8, 128, 33),
+                                       (2, 1, 256, 5)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_nested_attention_is_softmax_attention_on_the_dequantised_cache(oracle_mod, H, Hkv, D, T,
+                                                                       mode):
+    """numpy's softmax attention over the (separately pinned) dequantised
+    cache, heads grouped as h // (H / Hkv)."""
+    q, k, v = _kv_case(H + T, H, Hkv, D, T)
+    kp, vp = oracle_mod.kv_pack(k), oracle_mod.kv_pack(v)
+    K = oracle_mod.dequant(mode, kp[0], kp[1], kp[2], D).reshape(T, Hkv, D)
+    V = oracle_mod.dequant(mode, vp[0], vp[1], vp[2], D).reshape(T, Hkv, D)
+    ref = np.empty((H, D))
+    for h in range(H):
+        j = h // (H // Hkv)
+        sc = K[:, j, :] @ q[h].astype(np.float64) / np.sqrt(D)
+        p = np.exp(sc - sc.max())
+        ref[h] = (p / p.sum()) @ V[:, j, :]
+    got = oracle_mod.nested_attention(mode, q, kp, vp, Hkv)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_nested_attention_closed_forms(oracle_mod):
+    """One cached token: every head returns its KV head's value row.  A zero
+    query: uniform weights, the mean of the value rows."""
+    H, Hkv, D = 4, 2, 128
+    q, k, v = _kv_case(1, H, Hkv, D, 1)
+    kp, vp = oracle_mod.kv_pack(k), oracle_mod.kv_pack(v)
+    V = oracle_mod.dequant(1, vp[0], vp[1], vp[2], D)
+    out = oracle_mod.nested_attention(1, q, kp, vp, Hkv)
+    for h in range(H):
+        assert np.array_equal(out[h], V[h // 2])
+    T = 6
+    _, k, v = _kv_case(2, H, Hkv, D, T)
+    kp, vp = oracle_mod.kv_pack(k), oracle_mod.kv_pack(v)
+    V = oracle_mod.dequant(0, vp[0], None, vp[2], D).reshape(T, Hkv, D)
+    out = oracle_mod.nested_attention(0, np.zeros((H, D), np.float16), kp, vp, Hkv)
+    for h in range(H):
+        assert np.allclose(out[h], V[:, h // 2, :].mean(axis=0), rtol=1e-13, atol=1e-13)
+
+
+def test_nested_attention_draft_equals_target_when_lo_is_eight(oracle_mod):
+    H, Hkv, D, T = 8, 2, 128, 9
+    q, k, v = _kv_case(3, H, Hkv, D, T)
+    kp, vp = list(oracle_mod.kv_pack(k)), list(oracle_mod.kv_pack(v))
+    eight = oracle_mod.pack_plane(np.full((T * Hkv, D), 8, np.uint8))
+    kp[1], vp[1] = eight, eight
+    d = oracle_mod.nested_attention(0, q, kp, vp, Hkv)
+    t = oracle_mod.nested_attention(1, q, kp, vp, Hkv)
+    assert np.array_equal(d, t)
