@@ -619,6 +619,56 @@ def measure_hadamard(wl, hbm_peak, reps=20):
             "per_case": res}
 
 
+# ------------------------------------------ nested KV cache: decode attention
+def attention_bytes(mode, H, Hkv, T, D=128):
+    """Algorithmic bytes of one decode-attention launch: the K and V hi planes
+    (and lo planes for the target) and their fp16 row scales, the fp16 query,
+    the fp32 output."""
+    rows = T * Hkv
+    planes = (1 if mode == 0 else 2) * 2 * rows * (D // 2)
+    return planes + 2 * 2 * rows + 2 * H * D + 4 * H * D
+
+
+def measure_attention(wl, hbm_peak, reps=20):
+    """bitnest_nested_attention for one Llama-3-8B decode token (32 query
+    heads, 8 KV heads, head_dim 128) over caches of 2048 and 8192 tokens
+    (seeded synthetic K / V packed with bitnest_pack_weights), draft (KV4) and
+    target (KV8); one launch after a spin, CUDA events."""
+    import torch
+
+    bn = wl.bn
+    H, Hkv, D = 32, 8, 128
+    gen = torch.Generator(device=wl.dev)
+    gen.manual_seed(synth.SEED_ACTS + 700)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    res = {}
+    for T in (2048, 8192):
+        kv = [torch.randn((T * Hkv, D), generator=gen, device=wl.dev).half() for _ in range(2)]
+        kp, vp = bn.pack_weights(kv[0]), bn.pack_weights(kv[1])
+        q = torch.randn((H, D), generator=gen, device=wl.dev).half()
+        out = torch.empty((H, D), dtype=torch.float32, device=wl.dev)
+        for mode in (0, 1):
+            bn.nested_attention(mode, q, kp, vp, Hkv, out=out)
+            t = 0.0
+            for _ in range(reps):
+                torch.cuda._sleep(200_000)
+                a.record()
+                bn.nested_attention(mode, q, kp, vp, Hkv, out=out)
+                b.record()
+                torch.cuda.synchronize()
+                t += a.elapsed_time(b) / 1e3
+            t /= reps
+            nb = attention_bytes(mode, H, Hkv, T, D)
+            res[f"{'draft' if mode == 0 else 'target'}/T={T}"] = {
+                "us": round(t * 1e6, 2), "GB/s": round(nb / t / 1e9, 1),
+                "frac_hbm": round(nb / t / 1e9 / hbm_peak, 3)}
+        del kv, kp, vp
+    return {"workload": "decode attention of one token over a nested KV cache (H=32, Hkv=8, "
+                        "D=128), draft reads KV4 (hi planes), target KV8 (hi + lo)",
+            "per_case": res}
+
+
 # ------------------------------------------------ packer from fp weights
 def measure_pack(wl, hbm_peak, reps=5):
     """bitnest_pack_weights on the seven projections' shapes (seeded
@@ -747,7 +797,8 @@ def main():
                     help="launch the step's kernels directly instead of replaying a CUDA graph "
                          "(for profilers that cannot replay the captured kernel nodes)")
     ap.add_argument("--workload", default="all",
-                    choices=["all", "decode", "prefill", "sweep", "round", "pack", "hadamard"],
+                    choices=["all", "decode", "prefill", "sweep", "round", "pack", "hadamard",
+                             "attention"],
                     help="all: the decode step line with the prefill, M-sweep and "
                          "decode-round objects; otherwise only that part (profiling runs)")
     args = ap.parse_args()
@@ -794,6 +845,12 @@ def main():
     had = None
     if args.workload in ("all", "hadamard"):
         had = measure_hadamard(wl, hbm_peak)
+    att = None
+    if args.workload in ("all", "attention"):
+        try:  # an auxiliary row: its failure must not cost the step's line
+            att = measure_attention(wl, hbm_peak)
+        except Exception as e:  # noqa: BLE001
+            att = {"error": f"{type(e).__name__}: {e}"}
     prefill = None
     if args.workload in ("all", "prefill"):
         pre, pre_ops, pre_t = measure_prefill(wl, reps=10 if args.workload == "all" else 3)
@@ -815,7 +872,8 @@ def main():
             dist.destroy_process_group()
         if rank == 0:
             part = {"prefill": prefill, "m_sweep": sweep, "decode_round": rnd,
-                    "pack_from_weights": pack, "down_proj_input_rotation": had}
+                    "pack_from_weights": pack, "down_proj_input_rotation": had,
+                    "nested_kv_attention": att}
             print(json.dumps({"metric": METRIC, "workload": f"{args.workload} only",
                               **{k: v for k, v in part.items() if v is not None}}), flush=True)
         return
@@ -856,6 +914,8 @@ def main():
         out["pack_from_weights"] = pack
     if had is not None:
         out["down_proj_input_rotation"] = had
+    if att is not None:
+        out["nested_kv_attention"] = att
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, cores, rows = cpu_baseline()
         out["cpu_baseline"] = {

@@ -142,6 +142,29 @@ int bitnest_hadamard_quantize_act(const uint16_t *x, int64_t M, int64_t K, int8_
                                   float *xscale, int32_t *xsum, void *stream);
 
 /*
+ * Decode attention of one new token over a nested KV cache (model card,
+ * model table row "KV cache": nested at runtime, the draft reads KV4, the
+ * target KV8).  The card does not give the cache layout; this library's
+ * reading is the weights' nesting: each K (V) row of one token and one KV
+ * head, D = 128 values, is packed by bitnest_pack_weights (planes and one
+ * fp16 scale per row); the draft dequantises (hi - 8) s and reads only the
+ * hi planes, the target (16 (hi - 8) + (lo - 8)) s / 16.
+ *   q                   : fp16 [H, D], the new token's query heads.
+ *   k_hi, k_lo, v_hi, v_lo : uint8 [T * Hkv, D/2] planes, row t * Hkv + j
+ *                         = token t, KV head j (lo planes only for TARGET).
+ *   k_scale, v_scale    : fp16 [T * Hkv, D/128] = [T * Hkv, 1].
+ *   out                 : fp32 [H, D];  head h attends with KV head
+ *                         h / (H / Hkv):  softmax(q K^T / sqrt(D)) V.
+ * D must be 128, H / Hkv one of 1, 2, 4, 8, T >= 1 (else
+ * BITNEST_ERR_UNSUPPORTED_SHAPE).  fp32 arithmetic: agrees with an exact
+ * evaluation to fp32 rounding.
+ */
+int bitnest_nested_attention(int mode, const uint16_t *q, int64_t H, int64_t Hkv, int64_t D,
+                             int64_t T, const uint8_t *k_hi, const uint8_t *k_lo,
+                             const uint16_t *k_scale, const uint8_t *v_hi, const uint8_t *v_lo,
+                             const uint16_t *v_scale, float *out, void *stream);
+
+/*
  * Pack unpacked nibbles into the planes of the model card's layout
  * ("Files": byte j holds column 2j in its low nibble, 2j+1 in its high).
  *   uh, ul : uint8 [N, K] nibble values; only the low 4 bits are used.

@@ -184,3 +184,22 @@ def test_hadamard_quantize_argument_checks(L):
     assert L.bitnest_hadamard_quantize_act(None, 2, 14336, v(A), v(A), None, None) == 1
     assert L.bitnest_hadamard_quantize_act(v(A), 2, 14336, v(MIS), v(A), None, None) == 3
     assert L.bitnest_hadamard_quantize_act(v(A), 0, 14336, None, None, None, None) == 0
+
+
+def test_nested_attention_argument_checks(L):
+    v = ctypes.c_void_p
+
+    def call(mode=1, H=32, Hkv=8, D=128, T=10, lo=A, q=A, out=A):
+        return L.bitnest_nested_attention(mode, v(q) if q else None, H, Hkv, D, T, v(A),
+                                          v(lo) if lo else None, v(A), v(A),
+                                          v(lo) if lo else None, v(A), v(out) if out else None,
+                                          None)
+
+    assert call(mode=2) == 1
+    assert call(D=64) == 2
+    assert call(H=24, Hkv=8) == 2  # 3 query heads per KV head
+    assert call(H=30, Hkv=8) == 2
+    assert call(T=0) == 2
+    assert call(q=0) == 1
+    assert call(lo=0) == 1  # the target needs the lo planes
+    assert call(out=MIS) == 3

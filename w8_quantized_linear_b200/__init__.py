@@ -57,6 +57,7 @@ def lib() -> ctypes.CDLL:
     L.bitnest_debug_wait_probe.restype = I
     L.bitnest_pack_weights.argtypes = [P, I64, I64, P, P, P, P]
     L.bitnest_hadamard_quantize_act.argtypes = [P, I64, I64, P, P, P, P]
+    L.bitnest_nested_attention.argtypes = [I, P, I64, I64, I64, I64, P, P, P, P, P, P, P, P]
     L.bitnest_quantize_act.argtypes = [P, I64, I64, I, P, P, P, P]
     L.bitnest_act_group_sums.argtypes = [P, I64, I64, P, P]
     L.bitnest_linear.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, P]
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
     L.bitnest_linear_ws_bytes.restype = I64
     for name in ("bitnest_pack_planes", "bitnest_pack_weights", "bitnest_quantize_act",
                  "bitnest_act_group_sums", "bitnest_hadamard_quantize_act",
+                 "bitnest_nested_attention",
                  "bitnest_linear", "bitnest_linear_path", "bitnest_select_path",
                  "bitnest_debug_group_sums", "bitnest_quantize_linear", "bitnest_linear_ws",
                  "bitnest_linear_static_ws"):
@@ -175,6 +177,23 @@ def hadamard_quantize_act(x, out=None):
     _check(lib().bitnest_hadamard_quantize_act(_ptr(x), M, K, _ptr(xq), _ptr(xs), _ptr(xsum),
                                                _stream(x)), "bitnest_hadamard_quantize_act")
     return xq, xs, xsum
+
+
+def nested_attention(mode: int, q, k_planes, v_planes, Hkv: int, out=None):
+    """Decode attention of one token over a nested KV cache: q fp16 [H, 128];
+    k_planes / v_planes = pack_weights(rows [T * Hkv, 128]); fp32 [H, 128]."""
+    import torch
+
+    H, D = q.shape
+    k_hi, k_lo, k_sc = k_planes
+    v_hi, v_lo, v_sc = v_planes
+    T = k_hi.shape[0] // Hkv
+    o = out if out is not None else torch.empty((H, D), dtype=torch.float32, device=q.device)
+    _check(lib().bitnest_nested_attention(int(mode), _ptr(q), H, int(Hkv), D, T, _ptr(k_hi),
+                                          _ptr(k_lo), _ptr(k_sc), _ptr(v_hi), _ptr(v_lo),
+                                          _ptr(v_sc), _ptr(o), _stream(q)),
+           "bitnest_nested_attention")
+    return o
 
 
 def act_group_sums(xq, out=None):

@@ -142,6 +142,24 @@ int bitnest_hadamard_quantize_act(const uint16_t *x, int64_t M, int64_t K, int8_
   return cuda_status(launch_hadamard_quantize(x, M, K, xq, xscale, xsum, (cudaStream_t)stream));
 }
 
+int bitnest_nested_attention(int mode, const uint16_t *q, int64_t H, int64_t Hkv, int64_t D,
+                             int64_t T, const uint8_t *k_hi, const uint8_t *k_lo,
+                             const uint16_t *k_scale, const uint8_t *v_hi, const uint8_t *v_lo,
+                             const uint16_t *v_scale, float *out, void *stream) {
+  if (mode != BITNEST_DRAFT && mode != BITNEST_TARGET) return BITNEST_ERR_INVALID_ARG;
+  if (!nested_attention_supported(H, Hkv, D, T)) return BITNEST_ERR_UNSUPPORTED_SHAPE;
+  if (!q || !k_hi || !k_scale || !v_hi || !v_scale || !out) return BITNEST_ERR_INVALID_ARG;
+  if (mode == BITNEST_TARGET && (!k_lo || !v_lo)) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(q) || misaligned(k_hi) || misaligned(k_scale) || misaligned(v_hi) ||
+      misaligned(v_scale) || misaligned(out) ||
+      (mode == BITNEST_TARGET && (misaligned(k_lo) || misaligned(v_lo))))
+    return BITNEST_ERR_MISALIGNED;
+  return cuda_status(launch_nested_attention(mode, q, H, Hkv, T, k_hi,
+                                             mode == BITNEST_TARGET ? k_lo : nullptr, k_scale,
+                                             v_hi, mode == BITNEST_TARGET ? v_lo : nullptr,
+                                             v_scale, out, (cudaStream_t)stream));
+}
+
 int bitnest_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
                            void *stream) {
   int s = check_shape(M, 0, K);

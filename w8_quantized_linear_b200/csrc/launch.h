@@ -34,6 +34,13 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t M, int64_t K, int act_gro
                             float *xs, int32_t *xsum, cudaStream_t st);
 cudaError_t launch_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
                                   cudaStream_t st);
+// Decode attention over a nested KV cache (D = 128, H / Hkv in {1,2,4,8}).
+bool nested_attention_supported(int64_t H, int64_t Hkv, int64_t D, int64_t T);
+cudaError_t launch_nested_attention(int mode, const uint16_t *q, int64_t H, int64_t Hkv,
+                                    int64_t T, const uint8_t *k_hi, const uint8_t *k_lo,
+                                    const uint16_t *k_scale, const uint8_t *v_hi,
+                                    const uint8_t *v_lo, const uint16_t *v_scale, float *out,
+                                    cudaStream_t st);
 // Hadamard rotation x H / sqrt(K) + per-token quantisation (K = p or 28 p,
 // p a power of two, K <= 32768).
 bool hadamard_supported(int64_t K);
