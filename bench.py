@@ -845,12 +845,6 @@ def main():
     had = None
     if args.workload in ("all", "hadamard"):
         had = measure_hadamard(wl, hbm_peak)
-    att = None
-    if args.workload in ("all", "attention"):
-        try:  # an auxiliary row: its failure must not cost the step's line
-            att = measure_attention(wl, hbm_peak)
-        except Exception as e:  # noqa: BLE001
-            att = {"error": f"{type(e).__name__}: {e}"}
     prefill = None
     if args.workload in ("all", "prefill"):
         pre, pre_ops, pre_t = measure_prefill(wl, reps=10 if args.workload == "all" else 3)
@@ -867,6 +861,13 @@ def main():
             "per_projection": pre,
             "l2": "flushed (256 MB write) before every timed launch",
         }
+    att = None
+    if args.workload in ("all", "attention"):
+        # an auxiliary row, measured last: its failure must not cost the rest
+        try:
+            att = measure_attention(wl, hbm_peak)
+        except Exception as e:  # noqa: BLE001
+            att = {"error": f"{type(e).__name__}: {e}"}
     if dec is None:
         if world > 1:
             dist.destroy_process_group()
