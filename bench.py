@@ -58,14 +58,16 @@ def linear_bytes(mode, M, N, K):
 
 
 def quant_bytes(M, K, act_group):
+    """fp16 activations read; int8 codes and their fp32 scales written."""
     G = K // 128
-    return 2 * M * K + M * K + 4 * (M if act_group == 0 else M * G) + 4 * M * G
+    return 2 * M * K + M * K + 4 * (M if act_group == 0 else M * G)
 
 
 def fused_bytes(mode, M, N, K, act_group):
-    """Algorithmic bytes of one quantise + linear call (bitnest_quantize_linear):
-    planes, fp16 group scales, fp16 activations read; int8 codes, their scales
-    and group sums, and the fp32 output written."""
+    """Algorithmic bytes of one quantise + linear call (bitnest_quantize_linear
+    without an xsum buffer: the layer forms the group sums itself): planes,
+    fp16 group scales, fp16 activations read; int8 codes, their scales and
+    the fp32 output written."""
     G = K // 128
     planes = (1 if mode == 0 else 2) * N * K // 2
     return planes + 2 * N * G + quant_bytes(M, K, act_group) + 4 * M * N
@@ -256,7 +258,6 @@ class DecodeWorkload:
         return dict(
             xq=torch.empty((M, K), dtype=torch.int8, device=self.dev),
             xs=torch.empty((M,) if g == 0 else (M, G), dtype=torch.float32, device=self.dev),
-            xsum=torch.empty((M, G), dtype=torch.int32, device=self.dev),
             y=torch.empty((M, N), dtype=torch.float32, device=self.dev),
             y_host=torch.empty((M, N), dtype=torch.float32).pin_memory(),
         )
@@ -295,7 +296,7 @@ class DecodeWorkload:
                 if events is not None:
                     events[gname, mode][0].record()
                 bn.quantize_linear(mode, hi, lo, s, x, g, out=b["y"],
-                                   act_out=(b["xq"], b["xs"], b["xsum"]), path=self._path())
+                                   act_out=(b["xq"], b["xs"], None), path=self._path())
                 if events is not None:
                     events[gname, mode][1].record()
         if e2e:  # and every output back in one download
@@ -308,7 +309,7 @@ class DecodeWorkload:
         b = self.pbufs[name, mode]
         hi, lo, s = self.single[name]
         return lambda: bn.quantize_linear(mode, hi, lo, s, b["x"], g, out=b["y"],
-                                          act_out=(b["xq"], b["xs"], b["xsum"]),
+                                          act_out=(b["xq"], b["xs"], None),
                                           path=self._path())
 
 
@@ -757,7 +758,7 @@ def measure_round(wl, hbm_peak, reps=10):
                     b = wl.bufs[gname, mode]
                     hi, lo, s = lw[gname]
                     bn.quantize_linear(mode, hi, lo, s, wl.x[gname, mode], g, out=b["y"],
-                                       act_out=(b["xq"], b["xs"], b["xsum"]), path=path)
+                                       act_out=(b["xq"], b["xs"], None), path=path)
 
     graph = capture(one_round)
     for _ in range(3):

@@ -24,8 +24,8 @@ def test_quantise_plus_layer_bytes(mode, M, N, K, g):
     G = K // 128
     reads = [((N, K // 2), np.uint8)] * (1 if mode == 0 else 2)  # planes
     reads += [((N, G), np.float16), ((M, K), np.float16)]  # scales, activations
-    writes = [((M, K), np.int8), ((M,) if g == 0 else (M, G), np.float32), ((M, G), np.int32),
-              ((M, N), np.float32)]  # codes, their scales, group sums, y
+    writes = [((M, K), np.int8), ((M,) if g == 0 else (M, G), np.float32),
+              ((M, N), np.float32)]  # codes, their scales, y (no group sums: the layer forms them)
     assert bench.fused_bytes(mode, M, N, K, g) == _nbytes(*reads, *writes)
 
 

@@ -75,7 +75,11 @@ def test_linear_argument_checks(L):
     assert _lin(L, M=-1) == 2
     assert _lin(L, hi=0) == 1
     assert _lin(L, scale=0) == 1
-    assert _lin(L, xsum=0) == 1
+    # xsum is optional (the kernels form the group sums): a NULL xsum passes
+    # the checks, as the misaligned output shows (nothing is launched)
+    assert _lin(L, xsum=0, y=MIS) == 3
+    assert _lin(L, xsum=0, M=0) == 0
+    assert _lin(L, xsum=MIS) == 3
     assert _lin(L, y=0) == 1
     assert _lin(L, mode=1, lo=0) == 1
     assert _lin(L, mode=1, lo=MIS) == 3
@@ -106,6 +110,7 @@ def test_quantize_linear_argument_checks(L):
     assert q(x=MIS) == 3
     assert q(xq=0) == 1
     assert q(xsum=MIS) == 3
+    assert q(xsum=0, x=MIS) == 3  # a NULL xsum passes the checks (nothing launched)
     assert q(K=200) == 2
     assert q(g=7) == 1
     assert q(path=5) == 1
@@ -129,6 +134,8 @@ def test_quantize_pack_sum_argument_checks(L):
     assert L.bitnest_act_group_sums(v(A), 4, 256, None, None) == 1
     assert L.bitnest_act_group_sums(v(A), 0, 256, v(A), None) == 0
     assert L.bitnest_debug_group_sums(1, v(A), None, v(A), v(A), 1, 1, 128, v(A), 0, None) == 1
+    # debug sums without xsum: the checks pass it (misaligned S shows where they stop)
+    assert L.bitnest_debug_group_sums(1, v(A), v(A), v(A), None, 1, 1, 128, v(MIS), 0, None) == 3
     assert L.bitnest_debug_group_sums(0, v(A), None, v(A), v(A), 0, 1, 128, v(A), 0, None) == 0
 
 

@@ -298,3 +298,42 @@ def test_fused_layer_group_as_the_bench_launches_it(members):
         y_ref = oracle.linear(mode, hi_r, lo_r if mode else None, s[rows], q, xs_ref, K, g)
         assert oracle.max_normalised_error(host(y)[:, rows], y_ref) <= TOL
     assert bn.device_wait_timeout(reset=True) == 0
+
+
+# -------------------------------------------- without caller group sums
+@pytest.mark.parametrize("M,N,K", [(1, 37, 1024), (4, 300, 4096), (8, 130, 1024),
+                                   (3, 17, 14336), (5, 33, 384), (2, 2500, 2048)])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("act_group", [0, 128])
+def test_gemv_without_group_sums(M, N, K, mode, act_group):
+    """xsum = NULL (a caller holding only int8 codes): the decode GEMV forms
+    the per-(token, group) sums from the codes it stages.  Exact group sums,
+    y against the oracle, and the same bits as with the quantiser's sums."""
+    p = Problem(M, N, K, seed=5 * M + N + K, act_group=act_group)
+    y0 = bn.linear(mode, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, p.d_xsum, act_group,
+                   path=bn.PATH_GEMV)
+    y1 = bn.linear(mode, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, None, act_group,
+                   path=bn.PATH_GEMV)
+    S = bn.debug_group_sums(mode, p.d_hi, p.d_lo, p.d_xq, None, path=bn.PATH_GEMV)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    assert oracle.max_normalised_error(host(y1), p.y_ref(mode)) <= TOL
+    assert np.array_equal(host(S), oracle.group_sums(mode, p.hi, p.lo, p.q, K))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 300, 4096), (4, 200, 14336), (12, 130, 1024),
+                                   (40, 300, 1152)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_quantize_linear_without_group_sums(M, N, K, mode):
+    """The one-call entry with no xsum buffer: codes and scales bit-exact,
+    y against the oracle on the GEMV and the tensor-core paths."""
+    p = Problem(M, N, K, seed=3 * M + N)
+    xq = torch.empty((M, K), dtype=torch.int8, device=DEV)
+    xs = torch.empty((M,), dtype=torch.float32, device=DEV)
+    for path in (bn.PATH_AUTO | bn.PATH_OVERLAP, bn.PATH_TC):
+        y, _ = bn.quantize_linear(mode, p.d_hi, p.d_lo, p.d_s, p.d_x, act_out=(xq, xs, None),
+                                  path=path)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(xq), p.q) and np.array_equal(host(xs), p.xs)
+        assert oracle.max_normalised_error(host(y), p.y_ref(mode)) <= TOL
+    assert bn.device_wait_timeout(reset=True) == 0

@@ -32,7 +32,7 @@ def _no_wait_timeouts():
 
 SHAPES = [(1, 1, 128), (9, 100, 256), (16, 128, 1024), (17, 129, 384), (33, 300, 1152),
           (64, 256, 512), (100, 200, 4096), (128, 128, 128), (129, 257, 1024),
-          (300, 130, 640)]
+          (300, 130, 640), (512, 128, 256), (520, 300, 384), (1000, 129, 1152)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -208,3 +208,67 @@ def test_tc_split_k_scratch_shared_by_shapes():
             torch.cuda.synchronize()
             assert torch.equal(y, y0), (rnd, p.M, p.N, p.K)
     assert int(torch.count_nonzero(shared[:8192])) == 0
+
+
+# ---------------------------------------------- without caller group sums
+XS_SHAPES = [(5, 37, 1024), (16, 128, 1024), (33, 300, 1152), (128, 257, 512),
+             (600, 300, 384), (1030, 150, 640)]
+
+
+@pytest.mark.parametrize("M,N,K", XS_SHAPES)
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("act_group", [0, 128])
+def test_tc_without_group_sums(M, N, K, mode, act_group):
+    """xsum = NULL: the tensor-core kernel forms each token's group sums from
+    the activation tile it loaded.  y equals the call with the quantiser's
+    sums bit for bit and the oracle within the bar; the exact group sums too."""
+    p = Problem(M, N, K, seed=13 * M + N, act_group=act_group)
+    y0 = bn.linear(mode, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, p.d_xsum, act_group,
+                   path=bn.PATH_TC)
+    y1 = bn.linear(mode, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, None, act_group, path=bn.PATH_TC)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    assert oracle.max_normalised_error(host(y1), p.y_ref(mode)) <= TOL
+    if act_group == 0:
+        S = bn.debug_group_sums(mode, p.d_hi, p.d_lo, p.d_xq, None, path=bn.PATH_TC)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(S), oracle.group_sums(mode, p.hi, p.lo, p.q, K))
+
+
+def test_tc_split_k_without_group_sums():
+    """Split K and no caller sums together, on caller scratch."""
+    M, N, K = 16, 300, 1024
+    p = Problem(M, N, K, seed=8)
+    for mode in (0, 1):
+        ws = bn.workspace(bn.linear_ws_bytes(mode, M, N, K, bn.PATH_TC), DEV)
+        y = bn.linear_ws(mode, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, None, ws, path=bn.PATH_TC)
+        torch.cuda.synchronize()
+        assert oracle.max_normalised_error(host(y), p.y_ref(mode)) <= TOL
+        assert int(torch.count_nonzero(ws[:8192])) == 0
+
+
+def test_llama3_gate_prefill_without_group_sums():
+    """gate_proj at M = 2048 (tiles of 256 tokens) with xsum = NULL: the
+    same bits as with the quantiser's sums; sampled outputs against the oracle."""
+    name = "gate_proj"
+    N, K, act_group = synth.LLAMA3_8B_PROJECTIONS[name]
+    M = 2048
+    pid = synth.PROJ_IDS[name]
+    uh = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K)
+    ul = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K)
+    s = synth.group_scales(synth.SEED_SCALES + pid, N, K)
+    x = synth.activations(synth.SEED_ACTS + pid + 1, M, K)
+    d_hi, d_lo = bn.pack_planes(dev(uh), dev(ul))
+    d_s = dev(s)
+    d_xq, d_xs, d_xsum = bn.quantize_act(dev(x), act_group)
+    y0 = bn.linear(1, d_hi, d_lo, d_s, d_xq, d_xs, d_xsum, act_group)
+    y1 = bn.linear(1, d_hi, d_lo, d_s, d_xq, d_xs, None, act_group)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    rng = np.random.default_rng(pid + 1)
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.choice(N, 40, replace=False)]))
+    toks = np.unique(np.concatenate([[0, 255, 256, M - 1], rng.choice(M, 20, replace=False)]))
+    q, xs = oracle.quantize(x, act_group)
+    y_ref = oracle.linear(1, oracle.pack_plane(uh[rows]), oracle.pack_plane(ul[rows]), s[rows],
+                          q[toks], xs[toks], K, act_group)
+    assert oracle.max_normalised_error(host(y1)[np.ix_(toks, rows)], y_ref) <= TOL

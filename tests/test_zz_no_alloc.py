@@ -20,6 +20,15 @@ if not torch.cuda.is_available():  # pragma: no cover
 from test_gpu_parity import DEV, Problem, host  # noqa: E402
 
 
+@pytest.fixture(scope="module", autouse=True)
+def _no_earlier_timeout():
+    """The static scratch is shared by the whole process: start only from a
+    clean state (no bounded wait has given up, so no split call has left
+    arrivals behind), which a failure here would otherwise be blamed on."""
+    assert bn.device_wait_timeout() == 0
+    yield
+
+
 @pytest.mark.parametrize("M,N,K,path", [(16, 300, 1024, bn.PATH_TC), (1, 100, 4096, bn.PATH_TC),
                                         (128, 256, 14336, bn.PATH_TC),
                                         (8, 4096, 14336, bn.PATH_AUTO)])
@@ -68,3 +77,21 @@ def test_static_scratch_shared_by_shapes():
             y0 = bn.linear_ws(*args, ws, path=bn.PATH_TC)
             torch.cuda.synchronize()
             assert torch.equal(y, y0), (rnd, p.M, p.N, p.K)
+
+
+def test_static_scratch_back_to_back_with_programmatic_launch():
+    """Several static-scratch calls of different split shapes in a row on one
+    stream, with programmatic dependent launch and no synchronisation between
+    them: each y equals the caller-scratch result, and no wait gave up."""
+    shapes = [(16, 300, 1024), (128, 256, 14336), (8, 4096, 14336), (33, 129, 2048)]
+    probs = [Problem(M, N, K, seed=3 * M + K) for M, N, K in shapes]
+    path = bn.PATH_TC | bn.PATH_OVERLAP
+    ys = [bn.linear_static_ws(1, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, p.d_xsum, path=path)
+          for p in probs for _ in range(2)]
+    torch.cuda.synchronize()
+    for i, p in enumerate(probs):
+        ws = bn.workspace(bn.linear_ws_bytes(1, p.M, p.N, p.K, bn.PATH_TC), DEV)
+        y0 = bn.linear_ws(1, p.d_hi, p.d_lo, p.d_s, p.d_xq, p.d_xs, p.d_xsum, ws, path=bn.PATH_TC)
+        torch.cuda.synchronize()
+        assert torch.equal(ys[2 * i], y0) and torch.equal(ys[2 * i + 1], y0), (p.M, p.N, p.K)
+    assert bn.device_wait_timeout(reset=True) == 0

@@ -32,10 +32,10 @@ int check_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t 
   int s = check_shape(M, N, K);
   if (s != BITNEST_OK) return s;
   if (M == 0 || N == 0) return BITNEST_OK;  // empty problem: pointers are not inspected
-  if (!hi || !scale || !xq || !xscale || !xsum || !y) return BITNEST_ERR_INVALID_ARG;
+  if (!hi || !scale || !xq || !xscale || !y) return BITNEST_ERR_INVALID_ARG;
   if (mode == BITNEST_TARGET && !lo) return BITNEST_ERR_INVALID_ARG;
   if (misaligned(hi) || misaligned(scale) || misaligned(xq) || misaligned(xscale) ||
-      misaligned(xsum) || misaligned(y) || (bias && misaligned(bias)) ||
+      (xsum && misaligned(xsum)) || misaligned(y) || (bias && misaligned(bias)) ||
       (mode == BITNEST_TARGET && misaligned(lo)))
     return BITNEST_ERR_MISALIGNED;
   return BITNEST_OK;
@@ -87,6 +87,12 @@ int bitnest_device_wait_timeout(int reset) {
   int f1 = 0, f2 = 0;
   if (read_wait_timeout(&f1, reset != 0) != cudaSuccess) return -BITNEST_ERR_CUDA;
   if (read_wait_timeout_gemv(&f2, reset != 0) != cudaSuccess) return -BITNEST_ERR_CUDA;
+  // a split call that gave up may have left arrivals in the counters of the
+  // library's static scratch: the reset clears them as well
+  if (reset && f1) {
+    if (tc_static_ws_clear_counters(nullptr) != cudaSuccess) return -BITNEST_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -BITNEST_ERR_CUDA;
+  }
   return (f1 | f2) ? 1 : 0;
 }
 
@@ -291,9 +297,8 @@ int bitnest_debug_group_sums(int mode, const uint8_t *hi, const uint8_t *lo,
   int s = check_shape(M, N, K);
   if (s != BITNEST_OK) return s;
   if (M == 0 || N == 0) return BITNEST_OK;
-  if (!hi || !xq || !xsum || !S || (mode == BITNEST_TARGET && !lo))
-    return BITNEST_ERR_INVALID_ARG;
-  if (misaligned(hi) || misaligned(xq) || misaligned(xsum) || misaligned(S) ||
+  if (!hi || !xq || !S || (mode == BITNEST_TARGET && !lo)) return BITNEST_ERR_INVALID_ARG;
+  if (misaligned(hi) || misaligned(xq) || (xsum && misaligned(xsum)) || misaligned(S) ||
       (mode == BITNEST_TARGET && misaligned(lo)))
     return BITNEST_ERR_MISALIGNED;
   if (M == 0 || N == 0) return BITNEST_OK;

@@ -62,7 +62,6 @@ struct Params {
   const uint16_t *scale;
   const int8_t *xq;
   const float *xscale;
-  const int32_t *xsum;
   const uint16_t *bias;
   float *y;
   int32_t *S;
@@ -276,13 +275,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   griddep_wait();  // the activations are written by the preceding kernel
   const int C = p.K / 32;
-  // activations and group sums: every load of this thread first (one round
-  // trip), then the permuted stores
+  // token slots M..7 of the group sums (the MMA's unused columns) are zero
+  if constexpr (M < 8)
+    for (int i = threadIdx.x; i < Gp * (8 - M); i += NT) sr[(i / (8 - M)) * 8 + M + i % (8 - M)] = 0;
+  // activations (and per-group activation scales): every load of this
+  // thread first (one round trip), then the permuted stores and the group
+  // sums, formed here from the codes themselves
   constexpr int XB = 8;  // activation items per batch
-  constexpr int RB = 4;  // group-sum items per batch
-  for (int bx = 0, br = 0; bx < M * Cp || br < Gp * 8; bx += XB * NT, br += RB * NT) {
+  constexpr int RB = 4;  // activation-scale items per batch
+  for (int bx = 0, br = 0; bx < M * Cp || (ACTG && br < Gp * 8); bx += XB * NT, br += RB * NT) {
     uint4 va[XB], vb[XB];
-    int rv[RB];
     float xv[RB];
 #pragma unroll
     for (int u = 0; u < XB; ++u) {
@@ -298,13 +300,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (ACTG) {
 #pragma unroll
-    for (int u = 0; u < RB; ++u) {
-      const int i = br + threadIdx.x + u * NT;
-      const int g = i >> 3, m = i & 7;
-      const bool in = i < Gp * 8 && m < M && g < G;
-      rv[u] = in ? __ldg(p.xsum + m * G + g) : 0;
-      xv[u] = (ACTG && in) ? __ldg(p.xscale + m * G + g) : 0.0f;
+      for (int u = 0; u < RB; ++u) {
+        const int i = br + threadIdx.x + u * NT;
+        const int g = i >> 3, m = i & 7;
+        const bool in = i < Gp * 8 && m < M && g < G;
+        xv[u] = in ? __ldg(p.xscale + m * G + g) : 0.0f;
+      }
     }
     if (bx == 0) {  // loads of the first batch issued: the weight stream may go on
       __syncwarp();
@@ -312,11 +315,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 #pragma unroll
     for (int u = 0; u < XB; ++u) {
+      // items bx + threadIdx.x + u NT: the four 32-column chunks of a group
+      // are four consecutive lanes (Cp and NT are multiples of 4), so every
+      // lane takes part in the shuffles below
       const int item = bx + threadIdx.x + u * NT;
+      const uint32_t w[8] = {va[u].x, va[u].y, va[u].z, va[u].w,
+                             vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+      int r = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) r = __dp4a((int)w[i], 0x01010101, r);
+      r += __shfl_xor_sync(0xffffffffu, r, 1);
+      r += __shfl_xor_sync(0xffffffffu, r, 2);
       if (item < M * Cp) {
         const int m = item / Cp, c = item - m * Cp;
-        const uint32_t w[8] = {va[u].x, va[u].y, va[u].z, va[u].w,
-                               vb[u].x, vb[u].y, vb[u].z, vb[u].w};
         uint32_t e[4], o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -325,14 +336,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         xs4[(m * 2 + 0) * Cp + c] = make_uint4(e[0], o[0], e[1], o[1]);
         xs4[(m * 2 + 1) * Cp + c] = make_uint4(e[2], o[2], e[3], o[3]);
+        if ((c & 3) == 0) sr[(c >> 2) * 8 + m] = r;  // group c / 4 of token m (0 past K)
       }
     }
+    if (ACTG) {
 #pragma unroll
-    for (int u = 0; u < RB; ++u) {
-      const int i = br + threadIdx.x + u * NT;
-      if (i < Gp * 8) {
-        sr[i] = rv[u];
-        if (ACTG) sxg[i] = xv[u];
+      for (int u = 0; u < RB; ++u) {
+        const int i = br + threadIdx.x + u * NT;
+        if (i < Gp * 8) sxg[i] = xv[u];
       }
     }
   }
@@ -509,7 +520,6 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   p.scale = a.scale;
   p.xq = a.xq;
   p.xscale = a.xscale;
-  p.xsum = a.xsum;
   p.bias = a.bias;
   p.y = a.y;
   p.S = a.S;

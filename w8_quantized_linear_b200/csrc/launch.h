@@ -13,7 +13,7 @@ struct LinearArgs {
   const uint16_t *scale;  // fp16 [N, K/128]
   const int8_t *xq;       // [M, K]
   const float *xscale;    // [M] or [M, K/128]
-  const int32_t *xsum;    // [M, K/128]
+  const int32_t *xsum;    // [M, K/128] or null (the kernels form the sums)
   const uint16_t *bias;   // fp16 [N] or null
   float *y;               // [M, N]
   int32_t *S;             // debug group sums [M, N, K/128] (null unless debug)
@@ -65,6 +65,8 @@ int64_t tc_ws_bytes(int64_t M, int64_t N, int64_t K);
 // static split-K scratch.
 constexpr int64_t kStaticWsBytes = int64_t(12) << 20;
 cudaError_t tc_static_ws(void **ws);
+// Zero the arrival counters of that scratch (after a bounded wait gave up).
+cudaError_t tc_static_ws_clear_counters(cudaStream_t st);
 
 // The flag a bounded wait sets when it gives up (synchronous read).
 cudaError_t read_wait_timeout(int *flag, bool reset);

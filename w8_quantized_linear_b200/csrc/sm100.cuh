@@ -45,19 +45,60 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after a
-// bounded number of polls (each poll may suspend the thread briefly), sets
-// g_wait_timeout and returns false; also returns false at once if another
-// wait of the grid already gave up.
-constexpr uint32_t kMaxPolls = 1u << 22;
+// try_wait that may suspend the thread for up to `ns` nanoseconds while the
+// phase is incomplete; a completing phase wakes it, so a long hint costs no
+// latency and saves the shared-memory traffic of tight polling.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete.  Gives up after
+// `limit_ns` nanoseconds of device time (the global timer), sets
+// g_wait_timeout and returns false; also returns false soon after another
+// wait of the grid gave up.
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far beyond any legitimate wait
+constexpr uint32_t kSuspendHintNs = 20000;
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          uint32_t max_polls = kMaxPolls) {
-  for (uint32_t i = 0; i < max_polls; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023u) == 1023u && *(volatile int *)&g_wait_timeout) return false;
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
+    if ((i & 7u) == 0u) {
+      if (*(volatile int *)&g_wait_timeout) return false;
+      if (global_timer_ns() - t0 > limit_ns) break;
+    }
   }
   atomicExch(&g_wait_timeout, 1);
   return false;
+}
+
+// Bounded wait that does not give up early when another wait of the grid has
+// given up: used before releasing a resource (tensor memory) that work
+// already issued may still be using.
+__device__ __forceinline__ bool mbar_wait_final(uint64_t *bar, uint32_t parity,
+                                                uint64_t limit_ns = kWaitLimitNs) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait_hint(bar, parity, kSuspendHintNs))
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicExch(&g_wait_timeout, 1);
+      return false;
+    }
+  return true;
 }
 
 // Every lane of the warp polls; the warp agrees on the outcome (so the warp
@@ -201,6 +242,54 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 32 lanes x 32-bit, x N columns, every word set to `v`: thread i of the warp
+// fills lane (base + i).  Asynchronous; tmem_st_wait() waits for it.
+template <int N>
+__device__ __forceinline__ void tmem_st_const(uint32_t taddr, uint32_t v);
+
+template <>
+__device__ __forceinline__ void tmem_st_const<8>(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(
+                   taddr),
+               "r"(v)
+               : "memory");
+}
+
+template <>
+__device__ __forceinline__ void tmem_st_const<16>(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+template <>
+__device__ __forceinline__ void tmem_st_const<32>(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Move registers between the warpgroups of a CTA: every warp of a warpgroup
+// executes the same one.  The CTA's pool is its launch allocation (threads x
+// registers per thread at launch); increases must fit what decreases freed.
+template <int R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
 }
 
 }  // namespace bitnest

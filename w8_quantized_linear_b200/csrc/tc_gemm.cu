@@ -6,32 +6,46 @@
 // Both are formed here as ONE unsigned byte per weight (hi, or (hi<<4)|lo)
 // so a single kind::i8 MMA (u8 weights x s8 activations -> s32) per 32
 // columns does the work; the constant offset (8 or 136) times the
-// activation group sum is folded into the drain.
+// activation group sum is removed in the drain.
 //
-// Tile: 128 weight rows (the MMA's M, TMEM lanes) x BT tokens (the MMA's N),
-// one 128-column group per pipeline stage.  The group scales differ per
-// (row, group), so the int32 accumulator of every group is drained from TMEM
-// and scaled in fp32 (the model card's per-group scale); four TMEM
-// accumulators let the drain of a group run while the MMAs of the next
-// three proceed.  Persistent: one CTA per SM walks the tiles (token tiles
-// fastest, so the CTAs of a wave share weight rows in L2) and every role
-// runs ahead into the next tile while the epilogue finishes the current one.
+// Tile: 128 weight rows (the MMA's M, TMEM lanes) x BT tokens (the MMA's N,
+// up to 256), one 128-column group per pipeline stage.  The group scales
+// differ per (row, group), so the int32 accumulator of every group is
+// drained from TMEM and scaled in fp32 (the model card's per-group scale);
+// two (BT = 256) or four TMEM accumulators let the drain of a group run
+// while the MMAs of the next proceed.
 //
-// Every input stream runs well ahead of the MMAs: the TMA ring carries the
-// activation tile and the plane tiles of a group per stage, and the
-// per-group constants (row scales, per-token offsets) are read eight groups
-// per round trip into a ring of their own.
+// The drain costs one packed fp32 subtract and one packed fma per two
+// elements and no integer work: every accumulator starts each group at the
+// bit pattern of 1.5 * 2^23 (written back by the drain right after it reads
+// the group out), so the MMA leaves the float 1.5 * 2^23 + sum(q * byte) in
+// TMEM exactly (|sum| < 2^22); subtracting c = 1.5 * 2^23 + offset * sum(q)
+// (one fp32 constant per token and group) gives the exact group sum.
 //
-// Warp roles (15 warps):
-//   0..3   plane -> byte operand (shared-memory planes -> swizzled K-major)
+// A weight tile's operand bytes are built once per group and used by all BT
+// tokens of the tile: at BT = 256 that transform costs a quarter of the
+// drain.  Persistent: one CTA per SM walks the tiles (token tiles fastest, so
+// the CTAs of a wave share weight rows in L2) and every role runs ahead into
+// the next tile while the epilogue finishes the current one.
+//
+// Warp roles (16 warps, four warpgroups):
+//   0..3   plane -> byte operand (shared-memory planes -> swizzled K-major);
+//          without caller group sums also the tokens' sums of the group
+//          (from the landed activation tile)
 //   4      TMA producer: activation tile (128-byte swizzle) and the hi / lo
 //          plane tiles of the group, one mbarrier per stage (this CTA only)
 //   5      TMEM owner and MMA issuer (one thread)
-//   6      per-group constants: row scales, magic - offset * activation group
-//          sum per token (and the per-group activation scale for o_proj)
-//   7..14  epilogue: TMEM -> registers, exact int -> fp32, scale, accumulate
+//   6      per-group constants: row scales, per-token constants c (and the
+//          per-group activation scales for o_proj)
+//   7      idle
+//   8..15  epilogue: TMEM -> registers -> fp32 running sums (two warps per
+//          TMEM lane quarter, half of the tokens each)
+// At BT = 256 the epilogue holds 128 running sums per thread: the other
+// warpgroups hand registers to it (setmaxnreg).
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -43,23 +57,33 @@ namespace tc {
 
 constexpr int BW = 128;  // weight rows per tile
 constexpr int kMaxStages = 8;
-constexpr int kAccBufs = 4;    // TMEM accumulators
-constexpr int kCSlots = 16;    // per-group constant slots
-constexpr int kCBatch = 8;     // groups of constants per round trip
 constexpr int kWarpXf0 = 0, kNumXf = 4;
 constexpr int kWarpTma = 4, kWarpMma = 5, kWarpPrep = 6;
-constexpr int kWarpEpi0 = 7, kNumEpi = 8;  // two epilogue warps per TMEM lane quarter
-constexpr int kWarps = 15;
+constexpr int kWarpEpi0 = 8, kNumEpi = 8;  // two epilogue warps per TMEM lane quarter
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-// 1.5 * 2^23: adding an integer |s| < 2^22 to this bit pattern gives the
-// float 1.5 * 2^23 + s exactly, so int -> float is one integer add.
-constexpr int kMagicI = 0x4B400000;
+// 1.5 * 2^23: its bit pattern plus an integer |s| < 2^22 is the float
+// 1.5 * 2^23 + s exactly
+constexpr uint32_t kMagicI = 0x4B400000u;
 constexpr float kMagicF = 12582912.0f;
+// registers per thread of each warpgroup (sums to 512 threads x 128
+// registers, the launch allocation)
+constexpr int kRegXf = 48, kRegMisc = 96, kRegEpi = 184;
+static_assert(128 * kRegXf + 128 * kRegMisc + 256 * kRegEpi == kThreads * 128, "register pool");
+
+template <int BT>
+struct Cfg {
+  static constexpr int NACC = BT >= 256 ? 2 : 4;      // TMEM accumulators
+  static constexpr int CSLOTS = BT >= 256 ? 8 : 16;   // per-group constant slots
+  static constexpr int CBATCH = BT >= 128 ? 2 : 4;    // groups of constants per round trip
+  static constexpr int COLS = BT / 2;                 // tokens per epilogue warp
+  static constexpr int CH = COLS < 16 ? COLS : 16;    // columns per TMEM load
+};
 
 struct Params {
   const uint16_t *scale;   // fp16 [N, G]
   const float *xscale;     // [M] or [M, G]
-  const int32_t *xsum;     // [M, G]
+  const int32_t *xsum;     // [M, G] (unused when the kernel forms the sums)
   const uint16_t *bias;    // [N] or null
   float *y;                // [M, N]
   int32_t *S;              // debug sums [M, N, G]
@@ -93,9 +117,12 @@ __device__ __forceinline__ TileCoord tile_coord(const Params &p, int tile) {
 }
 
 __host__ __device__ constexpr int tmem_cols(int bt) {
-  // kAccBufs * bt rounded up to a power of two >= 32
-  return kAccBufs * bt <= 32 ? 32 : kAccBufs * bt <= 64 ? 64 : kAccBufs * bt <= 128 ? 128
-         : kAccBufs * bt <= 256 ? 256 : 512;
+  // accumulators x bt, rounded up to a power of two >= 32
+  return (bt >= 256 ? 2 : 4) * bt <= 32    ? 32
+         : (bt >= 256 ? 2 : 4) * bt <= 64  ? 64
+         : (bt >= 256 ? 2 : 4) * bt <= 128 ? 128
+         : (bt >= 256 ? 2 : 4) * bt <= 256 ? 256
+                                           : 512;
 }
 
 __host__ __device__ constexpr int stage_bytes(int mode, int bt) {
@@ -105,24 +132,18 @@ __host__ __device__ constexpr int stage_bytes(int mode, int bt) {
   return (BW * 128 + bt * 128 + (mode ? 2 : 1) * BW * 64 + 1023) / 1024 * 1024;
 }
 
-// one constant slot: row scales (128 fp32), column constants and activation
-// scales (bt x 4 B each)
+// one constant slot: row scales (128 fp32), per-token constants c and
+// activation scales (bt x 4 B each)
 __host__ __device__ constexpr int cslot_bytes(int bt) { return BW * 4 + 2 * bt * 4; }
 
+__host__ __device__ constexpr int cslots(int bt) { return bt >= 256 ? 8 : 16; }
+
 __host__ __device__ constexpr int smem_total(int mode, int bt, int stages) {
-  return 1024 + stages * stage_bytes(mode, bt) + kCSlots * cslot_bytes(bt) +
-         (3 * kMaxStages + 2 * kCSlots + 2 * kAccBufs) * 8 + 16;
+  return 1024 + stages * stage_bytes(mode, bt) + cslots(bt) * cslot_bytes(bt) +
+         (3 * kMaxStages + 2 * 16 + 2 * 4) * 8 + 16;
 }
 
-// d.{x,y} = a.{x,y} + b.{x,y} and d = a * b + c on float pairs (one packed
-// f32x2 instruction each).
-__device__ __forceinline__ void add2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 a, b, d;\n\t"
-      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
+// d = a * b + c on float pairs (one packed f32x2 instruction).
 __device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1,
                                      float c0, float c1) {
   asm("{\n\t.reg .b64 a, b, c, d;\n\t"
@@ -132,14 +153,15 @@ __device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
-template <int MODE, int BT, bool ACTG, bool DEBUG, bool SPLIT>
+// XS: the kernel forms the tokens' group sums itself (no caller xsum).
+template <int MODE, int BT, bool ACTG, bool DEBUG, bool SPLIT, bool XS>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_linear_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_hi,
                      const __grid_constant__ CUtensorMap tm_lo, const Params p) {
+  using C = Cfg<BT>;
   constexpr int OFF = CodeOffset<MODE>::value;
-  constexpr int COLS = BT / 2;               // columns per epilogue warp
-  constexpr int CH = COLS < 32 ? COLS : 32;  // columns per TMEM load
+  constexpr int NACC = C::NACC, CS = C::CSLOTS, COLS = C::COLS, CH = C::CH;
   constexpr uint32_t IDESC = umma_idesc_u8s8(BW, BT);
   constexpr int TCOLS = tmem_cols(BT);
   constexpr int STAGE = stage_bytes(MODE, BT);
@@ -148,26 +170,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  const int S = p.stages, G = p.G;
+  const int S = p.stages;
   // stage s: [A 16 KB][B bt x 128][hi 8 KB][lo 8 KB]
   auto sA = [&](int s) { return smem + s * STAGE; };
   auto sB = [&](int s) { return smem + s * STAGE + BW * 128; };
   auto sH = [&](int s) { return smem + s * STAGE + BW * 128 + BT * 128; };
   auto sL = [&](int s) { return smem + s * STAGE + BW * 128 + BT * 128 + BW * 64; };
-  // constant slot c: [row scales][column constants][act. scales]
+  // constant slot c: [row scales][per-token constants][act. scales]
   uint8_t *cbase = smem + S * STAGE;
   auto sSg = [&](int c) { return reinterpret_cast<float *>(cbase + c * CSLOT); };
-  auto sCv = [&](int c) { return reinterpret_cast<int32_t *>(sSg(c) + BW); };
-  auto sXv = [&](int c) { return reinterpret_cast<float *>(sCv(c) + BT); };
-  uint64_t *bars = reinterpret_cast<uint64_t *>(cbase + kCSlots * CSLOT);
+  auto sCv = [&](int c) { return sSg(c) + BW; };
+  auto sXv = [&](int c) { return sCv(c) + BT; };
+  uint64_t *bars = reinterpret_cast<uint64_t *>(cbase + CS * CSLOT);
   uint64_t *fullB = bars;                      // activation and plane tiles landed
   uint64_t *fullA = bars + kMaxStages;         // byte operand written
   uint64_t *stageFree = bars + 2 * kMaxStages; // MMAs done with the stage
-  uint64_t *fullC = bars + 3 * kMaxStages;     // [kCSlots] per-group constants written
-  uint64_t *emptyC = fullC + kCSlots;          // [kCSlots] epilogue done with them
-  uint64_t *accFull = emptyC + kCSlots;        // [kAccBufs] accumulator ready
-  uint64_t *accEmpty = accFull + kAccBufs;     // [kAccBufs] accumulator drained
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(accEmpty + kAccBufs);
+  uint64_t *fullC = bars + 3 * kMaxStages;     // [CS] per-group constants written
+  uint64_t *emptyC = fullC + CS;               // [CS] epilogue done with them
+  uint64_t *accFull = emptyC + CS;             // [NACC] accumulator ready
+  uint64_t *accEmpty = accFull + NACC;         // [NACC] accumulator drained and re-seeded
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(accEmpty + NACC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -177,11 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&fullA[s], kNumXf);
       mbar_init(&stageFree[s], 1);
     }
-    for (int c = 0; c < kCSlots; ++c) {
-      mbar_init(&fullC[c], 1);
+    for (int c = 0; c < CS; ++c) {
+      mbar_init(&fullC[c], XS ? 1 + kNumXf : 1);
       mbar_init(&emptyC[c], kNumEpi);
     }
-    for (int b = 0; b < kAccBufs; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(&accFull[b], 1);
       mbar_init(&accEmpty[b], kNumEpi);
     }
@@ -199,18 +221,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   // scales come from the preceding one (waited for below, before each read)
   griddep_launch_dependents();
 
+  // Each warpgroup's branch starts with its register count (the epilogue
+  // holds the fp32 running sums), so the compiler allocates every role
+  // within what it has.
   if (warp < kWarpXf0 + kNumXf) {
+    setmaxnreg_dec<kRegXf>();
     // ---------------------------------------------- plane -> operand bytes
     // thread t: rows pass * 32 + t / 4 (pass 0..3), 16-byte plane chunk
     // t % 4 of the group (32 columns) -> 32 operand bytes of that row
     const int t = threadIdx.x - kWarpXf0 * 32;  // 0..127
     const int qd = t & 3;
-    int s = 0;
+    int s = 0, it = 0;
     uint32_t ph = 0;  // stage slot and the parity of its current fill
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
       const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
-      for (int g = tc.g0; g < tc.g1; ++g) {
+      for (int g = tc.g0; g < tc.g1; ++g, ++it) {
         ok = mbar_wait_warp(&fullB[s], ph);
         if (!ok) break;
         const uint8_t *hs = sH(s);
@@ -246,15 +272,45 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_uint4(out[4], out[5], out[6], out[7]);
         }
         fence_proxy_async_smem();
+        int cs = 0;
+        if constexpr (XS) {
+          // the tokens' sums of this group from the landed activation tile
+          // (rows of 128 bytes in the 128-byte swizzle): eight threads per
+          // row, one 16-byte chunk each, c = 1.5 * 2^23 + offset * sum
+          cs = it % CS;
+          ok = mbar_wait_warp(&emptyC[cs], ((it / CS) & 1) ^ 1);
+          if (!ok) break;
+          float *cv = sCv(cs);
+          const uint8_t *bs = sB(s);
+          const int q = t & 7;
+#pragma unroll 4
+          for (int r0 = 0; r0 < BT; r0 += 16) {
+            const int r = r0 + (t >> 3);
+            const uint4 w = *reinterpret_cast<const uint4 *>(bs + r * 128 + ((q ^ (r & 7)) << 4));
+            int sum = __dp4a((int)w.x, 0x01010101, 0);
+            sum = __dp4a((int)w.y, 0x01010101, sum);
+            sum = __dp4a((int)w.z, 0x01010101, sum);
+            sum = __dp4a((int)w.w, 0x01010101, sum);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+            if (q == 0) cv[r] = kMagicF + (float)(OFF * sum);  // exact: |OFF * sum| < 2^22
+          }
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&fullA[s]);
+        if (lane == 0) {
+          mbar_arrive(&fullA[s]);
+          if (XS) mbar_arrive(&fullC[cs]);
+        }
         if (++s == S) {
           s = 0;
           ph ^= 1u;
         }
       }
     }
-  } else if (warp == kWarpTma) {
+  } else if (warp < kWarpEpi0) {
+    setmaxnreg_dec<kRegMisc>();
+    if (warp == kWarpTma) {
     // --------------------------------------------------------- TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -284,70 +340,75 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok)  // gave up: let the copies already issued land
-        for (int i = (it > S ? it - S : 0); i < it; ++i) mbar_wait(&fullB[i % S], (i / S) & 1);
+        for (int i = (it > S ? it - S : 0); i < it; ++i)
+          mbar_wait_final(&fullB[i % S], (i / S) & 1);
     }
-  } else if (warp == kWarpMma) {
+    } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       // every count, slot and descriptor is kept incrementally: this one
       // thread shares its scheduler with busy warps, so each instruction it
       // saves shortens the gap between two groups' MMAs
-      int s = 0, b = 0, it = 0;
-      uint32_t ph = 0, bph = 0;
+      int s = 0, b = 0, lb = 0;
+      uint32_t ph = 0, bph = 0, lbph = 0;
+      bool issued = false;
       const uint64_t ad0 = umma_desc_sw128(sA(0)), bd0 = umma_desc_sw128(sB(0));
       constexpr uint64_t kStageDesc = STAGE >> 4;  // descriptor address unit: 16 bytes
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
         const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
-        for (int g = tc.g0; g < tc.g1; ++g, ++it) {
-          ok = mbar_wait(&fullB[s], ph) && mbar_wait(&fullA[s], ph) &&
-               mbar_wait(&accEmpty[b], bph ^ 1u);
+        for (int g = tc.g0; g < tc.g1; ++g) {
+          // accEmpty[b] completes once per seeding of the accumulator: the
+          // epilogue seeds every accumulator once before the first group
+          ok = mbar_wait(&fullB[s], ph) && mbar_wait(&fullA[s], ph) && mbar_wait(&accEmpty[b], bph);
           if (!ok) break;
           tc_fence_after();
           const uint64_t ad = ad0 + (uint64_t)s * kStageDesc, bd = bd0 + (uint64_t)s * kStageDesc;
           const uint32_t dt = tmem + (uint32_t)(b * BT);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // 4 x K=32 bytes inside the 128-byte row
-            umma_i8(dt, ad + 2 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
+            umma_i8(dt, ad + 2 * kk, bd + 2 * kk, IDESC, 1u);  // onto the seed
           umma_commit(&stageFree[s]);
           umma_commit(&accFull[b]);
+          issued = true;
+          lb = b;
+          lbph = bph;
           if (++s == S) {
             s = 0;
             ph ^= 1u;
           }
-          if (++b == kAccBufs) {
+          if (++b == NACC) {
             b = 0;
             bph ^= 1u;
           }
         }
       }
-      // the last accumulator must be complete before TMEM is released
-      if (ok && it > 0) {
-        const int lb = b == 0 ? kAccBufs - 1 : b - 1;
-        mbar_wait(&accFull[lb], b == 0 ? bph ^ 1u : bph);
-      }
+      // every MMA issued must be complete before TMEM is released (also
+      // after a wait gave up): commits complete in order
+      if (issued) mbar_wait_final(&accFull[lb], lbph);
     }
-  } else if (warp == kWarpPrep) {
+    } else if (warp == kWarpPrep) {
     // ----------------------------------------------- per-group constants
-    // Eight groups per round trip: lane i holds rows i + 32 r (r < 4) and
+    // CBATCH groups per round trip: lane i holds rows i + 32 r (r < 4) and
     // tokens i + 32 u (u < BT / 32, at least one), all loads of a batch
     // issued before the first use.
     constexpr int TU = BT < 32 ? 1 : BT / 32;
+    constexpr int CB = C::CBATCH;
     griddep_wait();
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
       const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
-      const int n0 = tc.n0, m0 = tc.m0, G1 = tc.g1;
-      for (int gb = tc.g0; gb < G1 && ok; gb += kCBatch) {
-        uint16_t sv[4][kCBatch];
-        int rv[TU][kCBatch];
-        float xv[TU][kCBatch];
+      const int n0 = tc.n0, m0 = tc.m0, G1 = tc.g1, G = p.G;
+      for (int gb = tc.g0; gb < G1 && ok; gb += CB) {
+        uint16_t sv[4][CB];
+        int rv[TU][CB];
+        float xv[TU][CB];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int n = n0 + lane + 32 * r;
 #pragma unroll
-          for (int k = 0; k < kCBatch; ++k)
+          for (int k = 0; k < CB; ++k)
             sv[r][k] = (!DEBUG && n < p.N && gb + k < G1) ? __ldg(p.scale + (int64_t)n * G + gb + k)
                                                            : (uint16_t)0;
         }
@@ -356,20 +417,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int j = lane + 32 * u, m = m0 + j;
           const bool in = j < BT && m < p.M;
 #pragma unroll
-          for (int k = 0; k < kCBatch; ++k) {
-            rv[u][k] = (in && gb + k < G1) ? __ldg(p.xsum + (int64_t)m * G + gb + k) : 0;
+          for (int k = 0; k < CB; ++k) {
+            rv[u][k] = (!XS && in && gb + k < G1) ? __ldg(p.xsum + (int64_t)m * G + gb + k) : 0;
             xv[u][k] = (ACTG && in && gb + k < G1) ? __ldg(p.xscale + (int64_t)m * G + gb + k)
                                                    : 0.0f;
           }
         }
 #pragma unroll
-        for (int k = 0; k < kCBatch; ++k) {
+        for (int k = 0; k < CB; ++k) {
           if (gb + k >= G1) break;
-          const int c = it % kCSlots;
-          ok = mbar_wait_warp(&emptyC[c], ((it / kCSlots) & 1) ^ 1);
+          const int c = it % CS;
+          ok = mbar_wait_warp(&emptyC[c], ((it / CS) & 1) ^ 1);
           if (!ok) break;
           float *sg = sSg(c);
-          int32_t *cv = sCv(c);
+          float *cv = sCv(c);
           float *xs = sXv(c);
 #pragma unroll
           for (int r = 0; r < 4; ++r) sg[lane + 32 * r] = __half2float(__ushort_as_half(sv[r][k]));
@@ -377,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < TU; ++u) {
             const int j = lane + 32 * u;
             if (j < BT) {
-              cv[j] = kMagicI - OFF * rv[u][k];
+              if (!XS) cv[j] = kMagicF + (float)(OFF * rv[u][k]);  // exact
               if (ACTG) xs[j] = xv[u][k];
             }
           }
@@ -387,7 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    }
   } else {
+    setmaxnreg_inc<kRegEpi>();
     // -------------------------------------------------------------- epilogue
     const int e = warp - kWarpEpi0;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
@@ -395,45 +458,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;
     const int col0 = half * COLS;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    // seed every accumulator before its first group
+#pragma unroll
+    for (int b = 0; b < NACC; ++b)
+#pragma unroll
+      for (int c = 0; c < COLS; c += CH) tmem_st_const<CH>(tmem + lane_addr + b * BT + col0 + c, kMagicI);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0)
+      for (int b = 0; b < NACC; ++b) mbar_arrive(&accEmpty[b]);
     griddep_wait();  // y may still be read by the preceding kernel
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
       const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
       const int n = tc.n0 + row, m0 = tc.m0;
       float acc[COLS];
 #pragma unroll
       for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
       for (int g = tc.g0; g < tc.g1; ++g, ++it) {
-        const int cs = it % kCSlots, b = it % kAccBufs;
-        ok = mbar_wait_warp(&fullC[cs], (it / kCSlots) & 1) &&
-             mbar_wait_warp(&accFull[b], (it / kAccBufs) & 1);
-        if (!ok) break;
+        if (!ok) continue;  // after a give-up: no more waits, but every tile still arrives below
+        const int cs = it % CS, b = it % NACC;
+        ok = mbar_wait_warp(&fullC[cs], (it / CS) & 1) &&
+             mbar_wait_warp(&accFull[b], (it / NACC) & 1);
+        if (!ok) continue;
         tc_fence_after();
         const float sg = sSg(cs)[row];
-        const int32_t *cv = sCv(cs) + col0;
+        const float *cv = sCv(cs) + col0;
         const float *xv = sXv(cs) + col0;
 #pragma unroll
         for (int c = 0; c < COLS; c += CH) {
+          const uint32_t ta = tmem + lane_addr + b * BT + col0 + c;
           uint32_t d[CH];
-          tmem_ld<CH>(tmem + lane_addr + b * BT + col0 + c, d);
+          tmem_ld<CH>(ta, d);
           tmem_ld_wait();
+          tmem_st_const<CH>(ta, kMagicI);  // seed for the accumulator's next group
           if (DEBUG) {
 #pragma unroll
             for (int j = 0; j < CH; ++j) {
               const int m = m0 + col0 + c + j;
-              if (m < p.M && n < p.N)
-                p.S[((int64_t)m * p.N + n) * G + g] = (int)d[j] + cv[c + j] - kMagicI;
+              if (m < p.M && n < p.N)  // exact: both are integers of one binade
+                p.S[((int64_t)m * p.N + n) * p.G + g] =
+                    __float2int_rn(__int_as_float((int)d[j]) - cv[c + j]);
             }
           } else {
 #pragma unroll
             for (int j = 0; j < CH; j += 4) {
-              const int4 c4 = *reinterpret_cast<const int4 *>(cv + c + j);
-              // 1.5 * 2^23 + exact group sum, as a float, minus the magic
-              float f0 = __int_as_float((int)d[j] + c4.x), f1 = __int_as_float((int)d[j + 1] + c4.y);
-              float f2 = __int_as_float((int)d[j + 2] + c4.z), f3 = __int_as_float((int)d[j + 3] + c4.w);
-              add2(f0, f1, f0, f1, -kMagicF, -kMagicF);
-              add2(f2, f3, f2, f3, -kMagicF, -kMagicF);
+              const float4 c4 = *reinterpret_cast<const float4 *>(cv + c + j);
+              // 1.5 * 2^23 + raw sum, minus 1.5 * 2^23 + offset * sum(q): exact
+              float f0 = __int_as_float((int)d[j]), f1 = __int_as_float((int)d[j + 1]);
+              float f2 = __int_as_float((int)d[j + 2]), f3 = __int_as_float((int)d[j + 3]);
+              f32x2_sub(f0, f1, f0, f1, c4.x, c4.y);
+              f32x2_sub(f2, f3, f2, f3, c4.z, c4.w);
               float s0 = sg, s1 = sg, s2 = sg, s3 = sg;
               if (ACTG) {
                 const float4 x4 = *reinterpret_cast<const float4 *>(xv + c + j);
@@ -447,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -454,15 +532,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&emptyC[cs]);
         }
       }
-      if (SPLIT && !DEBUG && ok) {
+      if constexpr (SPLIT && !DEBUG) {
         // this range's partial sums of the warp's sub-block (rows of its lane
         // quarter, its columns), then one arrival per warp; the last of the
-        // splits to arrive adds them all in split order
+        // splits to arrive adds them all in split order.  A warp whose wait
+        // gave up still arrives (its partials are invalid, and so is y: the
+        // flag says so), so every counter returns to zero.
         float *part = p.ws + ((int64_t)tc.tmn * p.splits) * (BW * BT) + row * BT + col0;
+        if (ok) {
 #pragma unroll
-        for (int j = 0; j < COLS; j += 4)
-          *reinterpret_cast<float4 *>(part + (int64_t)tc.split * (BW * BT) + j) =
-              make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+          for (int j = 0; j < COLS; j += 4)
+            *reinterpret_cast<float4 *>(part + (int64_t)tc.split * (BW * BT) + j) =
+                make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+        }
         __threadfence();
         __syncwarp();
         int last = 0;
@@ -471,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!last) continue;
         __threadfence();
         if (lane == 0) p.cnt[tc.tmn * kNumEpi + e] = 0;  // ready for the next call
+        if (!ok) continue;
 #pragma unroll
         for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
         for (int sp = 0; sp < p.splits; ++sp) {
@@ -537,11 +620,14 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
+// Token tile: 256 from 512 tokens up (each transformed weight tile serves
+// twice the tokens; prefill), else the smallest of 16 .. 128 that holds M.
 int pick_bt(int64_t M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
-  return 128;
+  if (M < 512) return 128;
+  return 256;
 }
 
 int pick_stages(int mode, int bt, int max_smem) {
@@ -566,6 +652,7 @@ int num_sms() {
 // per epilogue warp and tile) at a fixed place, the start, so that calls of
 // any shapes can share one scratch (each leaves its counters zero, and no
 // shape's partial tiles reach another's counters); then the partial tiles.
+// Tiles of 256 tokens are never split.
 constexpr int kMaxCntTiles = 256;
 constexpr int64_t kCntBytes = int64_t(kMaxCntTiles) * kNumEpi * 4;  // 8 KB
 struct SplitPlan {
@@ -578,7 +665,7 @@ SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int bt) {
   sp.tmn = ((N + BW - 1) / BW) * ((M + bt - 1) / bt);
   const int sms = num_sms();
   int s = 1;
-  if (sp.tmn * 2 <= sms && sp.tmn <= kMaxCntTiles) {
+  if (bt <= 128 && sp.tmn * 2 <= sms && sp.tmn <= kMaxCntTiles) {
     s = (int)(sms / sp.tmn);
     if (s > G / 4) s = G / 4;
     if (s < 1) s = 1;
@@ -589,7 +676,18 @@ SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int bt) {
   return sp;
 }
 
-template <int MODE, int BT, bool ACTG, bool DEBUG>
+// The register split hands out exactly the launch allocation of 128
+// registers per thread; a kernel built with fewer would make the increase
+// wait for registers that do not exist, so it is not launched.
+template <typename Kern>
+cudaError_t check_register_pool(Kern kern) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  return fa.numRegs == 128 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+template <int MODE, int BT, bool ACTG, bool DEBUG, bool XS>
 cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   // split K only where the plan asks for it: the unsplit kernel carries none
   // of the partial-tile code
@@ -639,9 +737,12 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   p.stages = stages;
   const int grid = p.tiles < num_sms() ? p.tiles : num_sms();
   const int smem = smem_total(MODE, BT, stages);
-  auto kern = p.splits > 1 ? tc_linear_kernel<MODE, BT, ACTG, DEBUG, !DEBUG>
-                           : tc_linear_kernel<MODE, BT, ACTG, DEBUG, false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  constexpr bool kCanSplit = !DEBUG && BT <= 128;
+  auto kern = (kCanSplit && p.splits > 1) ? tc_linear_kernel<MODE, BT, ACTG, DEBUG, kCanSplit, XS>
+                                          : tc_linear_kernel<MODE, BT, ACTG, DEBUG, false, XS>;
+  cudaError_t e = check_register_pool(kern);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, a.overlap, mq, mh,
                  ml, p);
@@ -651,11 +752,15 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
 
 template <int MODE, int BT, bool DEBUG>
 cudaError_t launch_g(const LinearArgs &a, cudaStream_t st) {
+  const bool xs = a.xsum == nullptr;  // no caller sums: the kernel forms them
   // the debug sums take no activation scale: no per-group scale variant
   if constexpr (!DEBUG) {
-    if (a.act_group != 0) return launch_t<MODE, BT, true, false>(a, st);
+    if (a.act_group != 0)
+      return xs ? launch_t<MODE, BT, true, false, true>(a, st)
+                : launch_t<MODE, BT, true, false, false>(a, st);
   }
-  return launch_t<MODE, BT, false, DEBUG>(a, st);
+  return xs ? launch_t<MODE, BT, false, DEBUG, true>(a, st)
+            : launch_t<MODE, BT, false, DEBUG, false>(a, st);
 }
 
 template <int MODE, bool DEBUG>
@@ -664,16 +769,17 @@ cudaError_t launch_mode(const LinearArgs &a, cudaStream_t st) {
     case 16: return launch_g<MODE, 16, DEBUG>(a, st);
     case 32: return launch_g<MODE, 32, DEBUG>(a, st);
     case 64: return launch_g<MODE, 64, DEBUG>(a, st);
-    default: return launch_g<MODE, 128, DEBUG>(a, st);
+    case 128: return launch_g<MODE, 128, DEBUG>(a, st);
+    default: return launch_g<MODE, 256, DEBUG>(a, st);
   }
 }
 
 }  // namespace tc
 
-// Test hook: one warp waits, with the kernels' own bounded wait (cut to 4096
-// polls), on an mbarrier that nothing ever arrives at.  The wait gives up
-// and sets this translation unit's g_wait_timeout, which read_wait_timeout
-// reports; nothing faults or hangs.
+// Test hook: one warp waits, with the kernels' own bounded wait (cut to
+// 200 us of device time), on an mbarrier that nothing ever arrives at.  The
+// wait gives up and sets this translation unit's g_wait_timeout, which
+// read_wait_timeout reports; nothing faults or hangs.
 __global__ void wait_probe_kernel() {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
@@ -681,7 +787,7 @@ __global__ void wait_probe_kernel() {
     fence_barrier_init();
   }
   __syncwarp();
-  (void)mbar_wait(&bar, 0, 4096u);  // phase 0 never completes
+  (void)mbar_wait(&bar, 0, 200000ull);  // phase 0 never completes
 }
 
 cudaError_t launch_wait_probe(cudaStream_t st) {
@@ -708,21 +814,34 @@ bool tc_supported(int64_t M, int64_t N, int64_t K) {
 // counters: under 10 MB on 148 SMs.
 static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
 
+// Its device address, looked up once per device (the first caller on a
+// device does the lookup; the others wait for it).
 cudaError_t tc_static_ws(void **ws) {
+  static std::once_flag once[64];
   static void *addr[64] = {nullptr};
+  static cudaError_t err[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!addr[dev]) {  // once per device
+  std::call_once(once[dev], [dev] {
     void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_ws);
-    if (e != cudaSuccess) return e;
-    if (!p) return cudaErrorInvalidSymbol;
+    err[dev] = cudaGetSymbolAddress(&p, g_static_ws);
+    if (err[dev] == cudaSuccess && !p) err[dev] = cudaErrorInvalidSymbol;
     addr[dev] = p;
-  }
+  });
+  if (err[dev] != cudaSuccess) return err[dev];
   *ws = addr[dev];
   return cudaSuccess;
+}
+
+// After a bounded wait gave up inside a split call, the counters of the
+// static scratch may hold arrivals of that call: clear them (no allocation).
+cudaError_t tc_static_ws_clear_counters(cudaStream_t st) {
+  void *ws = nullptr;
+  cudaError_t e = tc_static_ws(&ws);
+  if (e != cudaSuccess) return e;
+  return cudaMemsetAsync(ws, 0, (size_t)tc::kCntBytes, st);
 }
 
 int64_t tc_ws_bytes(int64_t M, int64_t N, int64_t K) {
