@@ -78,18 +78,21 @@ const char *bitnest_status_string(int status);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int bitnest_version(void);
 
-/* Every wait of the tensor-core kernels on another warp or on a copy is
- * bounded; a wait that gives up sets a device flag and the kernel winds down
- * without finishing its output.  Returns that flag for the current device (1:
- * some launch since the last reset gave up, its outputs are invalid; 0: none),
- * or -BITNEST_ERR_CUDA.  Synchronous: reads device memory.  reset != 0 clears
- * the flag after reading it. */
+/* Every wait of the layer kernels on another warp or on a copy is bounded
+ * (a few seconds of device time); a wait that gives up sets a device flag and
+ * the kernel winds down without finishing its output.  Returns that flag for
+ * the current device (1: some launch since the last reset gave up, its
+ * outputs are invalid; 0: none), or -BITNEST_ERR_CUDA.  Synchronous: reads
+ * device memory.  reset != 0 clears the flag after reading it and, when it
+ * was set, also zeroes the arrival counters of the static split-K scratch
+ * (see bitnest_linear_static_ws).  A split-K call that gave up leaves the
+ * counters of caller scratch at zero as well: its warps still arrive. */
 int bitnest_device_wait_timeout(int reset);
 
 /* Test hook for the flag above: launches one warp that waits, with the
- * kernels' bounded wait (cut to 4096 polls), on an mbarrier that nothing
- * arrives at.  The wait gives up, sets the flag and the kernel returns;
- * nothing faults or hangs.  Asynchronous on `stream`; clear the flag with
+ * kernels' bounded wait (cut to 200 us of device time), on an mbarrier that
+ * nothing arrives at.  The wait gives up, sets the flag and the kernel
+ * returns; nothing faults or hangs.  Asynchronous on `stream`; clear the flag with
  * bitnest_device_wait_timeout(1) afterwards, or later bounded waits give up
  * at once. */
 int bitnest_debug_wait_probe(void *stream);
@@ -194,7 +197,8 @@ int bitnest_quantize_act(const uint16_t *x, int64_t M, int64_t K, int act_group,
 /*
  * Per-128-group sums of already quantised activations:
  *   xsum[m, g] = sum_{k in group g} xq[m, k]   (int32 [M, K/128]).
- * For callers whose xq does not come from bitnest_quantize_act.
+ * An optional input of the layer entry points (they form the sums
+ * themselves when given none).
  */
 int bitnest_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum,
                            void *stream);
@@ -207,11 +211,14 @@ int bitnest_act_group_sums(const int8_t *xq, int64_t M, int64_t K, int32_t *xsum
  *   scale     : fp16 [N, K/128] group scales.
  *   xq        : int8 [M, K] quantised activations.
  *   xscale    : fp32 [M] (act_group 0) or [M, K/128] (act_group 128).
- *   xsum      : int32 [M, K/128] group sums of xq (bitnest_quantize_act
- *               writes them).  Required: the tensor-core path folds the
- *               planes' unsigned-nibble offset (8 for hi, 136 for the
- *               combined byte) into one correction per (token, group) and
- *               takes it from here; it must match xq.
+ *   xsum      : int32 [M, K/128] group sums of xq, or NULL.  The kernels fold
+ *               the planes' unsigned-nibble offset (8 for hi, 136 for the
+ *               combined byte) into one correction per (token, group), which
+ *               needs these sums: the decode GEMV always forms them from the
+ *               codes it stages; the tensor-core path takes them from here
+ *               when given (they must match xq, as bitnest_quantize_act's
+ *               do) and otherwise forms them from the activation tiles it
+ *               loads.  The result is the same either way.
  *   y         : fp32 [M, N] output.
  *   bias      : fp16 [N] or NULL.
  * Integer group sums are exact (int32); the epilogue is fp32, so y agrees
@@ -243,8 +250,8 @@ int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const ui
  *                  bytes (BITNEST_ERR_INVALID_ARG if fewer).  When that is 0
  *                  ws may be NULL and the call is bitnest_linear_path.
  * The first 8 KB of ws hold arrival counters that must be zero before the
- * first call (cudaMemset once); every call leaves them zero, so one ws can
- * serve calls of any shapes.  Calls sharing one ws must not run at the same
+ * first call (cudaMemset once); every call leaves them zero, also one whose
+ * bounded wait gave up, so one ws can serve calls of any shapes.  Calls sharing one ws must not run at the same
  * time (calls in order on one stream are fine).
  * With BITNEST_PATH_AUTO the choice may differ from bitnest_select_path's:
  * where the TMA-ring GEMV does not apply and K would be split, the
@@ -260,10 +267,13 @@ int bitnest_linear_ws(int mode, const uint8_t *hi, const uint8_t *lo, const uint
  * bitnest_linear_ws without caller scratch and without any allocation: the
  * split-K partial sums and counters live in one file-scope static device
  * array of the library, BITNEST_STATIC_WS_BYTES (12 MiB) per device, zero
- * from module load and left zero by every call.  (The BitNest pages have no
- * counterpart to this entry point: it is a deployment convenience of this
- * library.)  The library calls no cudaMalloc / cudaFree here; it looks up the
- * array's device address once per device (cudaGetSymbolAddress) and caches it.
+ * from module load and left zero by every call (a call whose bounded wait
+ * gave up also leaves them zero; clearing the timeout flag zeroes them once
+ * more).  (The BitNest pages have no counterpart to this entry point: it is a
+ * deployment convenience of this library.)  The library calls no cudaMalloc /
+ * cudaFree here; the first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, once per device, thread-safe) and caches it.
+ * cudaDeviceReset unloads the module: the cached address is stale after it.
  *   - A problem whose split needs more than BITNEST_STATIC_WS_BYTES returns
  *     BITNEST_ERR_UNSUPPORTED_SHAPE, launching nothing.
  *   - Every call on a device shares the one array: calls that overlap in
@@ -292,7 +302,9 @@ int64_t bitnest_linear_ws_bytes(int mode, int64_t M, int64_t N, int64_t K, int p
  * bitnest_linear_path(mode, hi, lo, scale, xq, xscale, xsum, M, N, K, y,
  * act_group, bias, path), bit for bit in xq / xscale / xsum and y.
  *   x                 : fp16 [M, K] activations (finite values).
- *   xq, xscale, xsum  : outputs as in bitnest_quantize_act (all required).
+ *   xq, xscale        : outputs as in bitnest_quantize_act (required).
+ *   xsum              : output as in bitnest_quantize_act, or NULL (then not
+ *                       written, and the layer forms the sums itself).
  * The quantiser and the layer kernel run back to back on `stream`; with
  * BITNEST_PATH_OVERLAP the layer kernel streams its weights while the
  * quantiser runs.  Argument checks and
@@ -312,7 +324,8 @@ int bitnest_select_path(int mode, int64_t M, int64_t N, int64_t K);
  * Test hook: the exact int32 group sums the kernels of `path` form,
  *   S[m, n, g] = sum_{k in g} xq[m,k] * code[n,k],
  * code = hi - 8 (DRAFT) or 16*(hi - 8) + (lo - 8) (TARGET), written to
- * S int32 [M, N, K/128].  Same inner loops as bitnest_linear_path.
+ * S int32 [M, N, K/128].  Same inner loops as bitnest_linear_path; xsum as
+ * there (may be NULL).
  */
 int bitnest_debug_group_sums(int mode, const uint8_t *hi, const uint8_t *lo,
                              const int8_t *xq, const int32_t *xsum, int64_t M, int64_t N,

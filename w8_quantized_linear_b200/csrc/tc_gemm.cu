@@ -9,24 +9,24 @@
 // activation group sum is removed in the drain.
 //
 // Tile: 128 weight rows (the MMA's M, TMEM lanes) x BT tokens (the MMA's N,
-// up to 256), one 128-column group per pipeline stage.  The group scales
+// up to 128), one 128-column group per pipeline stage.  The group scales
 // differ per (row, group), so the int32 accumulator of every group is
 // drained from TMEM and scaled in fp32 (the model card's per-group scale);
-// two (BT = 256) or four TMEM accumulators let the drain of a group run
-// while the MMAs of the next proceed.
+// four TMEM accumulators let the drain of a group run while the MMAs of the
+// next three proceed.
 //
-// The drain costs one packed fp32 subtract and one packed fma per two
-// elements and no integer work: every accumulator starts each group at the
-// bit pattern of 1.5 * 2^23 (written back by the drain right after it reads
-// the group out), so the MMA leaves the float 1.5 * 2^23 + sum(q * byte) in
-// TMEM exactly (|sum| < 2^22); subtracting c = 1.5 * 2^23 + offset * sum(q)
-// (one fp32 constant per token and group) gives the exact group sum.
+// The drain turns each int32 group sum into fp32 exactly with one integer
+// add: the bit pattern of 1.5 * 2^23 minus offset * sum(q) (one constant per
+// token and group) plus the raw sum is the float 1.5 * 2^23 + exact group
+// sum (|sum| < 2^22); one packed subtract and one packed fma per two
+// elements finish it.  The drain reads a whole group out of TMEM, hands the
+// accumulator back to the MMA and only then does the arithmetic.
 //
-// A weight tile's operand bytes are built once per group and used by all BT
-// tokens of the tile: at BT = 256 that transform costs a quarter of the
-// drain.  Persistent: one CTA per SM walks the tiles (token tiles fastest, so
-// the CTAs of a wave share weight rows in L2) and every role runs ahead into
-// the next tile while the epilogue finishes the current one.
+// The drain reads each accumulator in 32-column chunks, the load of the next
+// chunk in flight while the current one is turned into fp32 sums.
+// Persistent: one CTA per SM walks the tiles (token tiles fastest, so the
+// CTAs of a wave share weight rows in L2) and every role runs ahead into the
+// next tile while the epilogue finishes the current one.
 //
 // Warp roles (16 warps, four warpgroups):
 //   0..3   plane -> byte operand (shared-memory planes -> swizzled K-major);
@@ -35,13 +35,12 @@
 //   4      TMA producer: activation tile (128-byte swizzle) and the hi / lo
 //          plane tiles of the group, one mbarrier per stage (this CTA only)
 //   5      TMEM owner and MMA issuer (one thread)
-//   6      per-group constants: row scales, per-token constants c (and the
-//          per-group activation scales for o_proj)
-//   7      idle
+//   6, 7   per-group constants, batches in turn: row scales, per-token
+//          constants c (and the per-group activation scales for o_proj)
 //   8..15  epilogue: TMEM -> registers -> fp32 running sums (two warps per
 //          TMEM lane quarter, half of the tokens each)
-// At BT = 256 the epilogue holds 128 running sums per thread: the other
-// warpgroups hand registers to it (setmaxnreg).
+// The other warpgroups hand registers to the epilogue (setmaxnreg), which
+// holds a tile row's running sums and a whole group of the accumulator.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -57,27 +56,34 @@ namespace tc {
 
 constexpr int BW = 128;  // weight rows per tile
 constexpr int kMaxStages = 8;
-constexpr int kWarpXf0 = 0, kNumXf = 4;
-constexpr int kWarpTma = 4, kWarpMma = 5, kWarpPrep = 6;
-constexpr int kWarpEpi0 = 8, kNumEpi = 8;  // two epilogue warps per TMEM lane quarter
-constexpr int kWarps = 16;
+constexpr int kWarpXf0 = 0, kNumXf = 4;  // one warpgroup
+constexpr int kXfThreads = 32 * kNumXf;
+constexpr int kXfPasses = 4 * 128 / kXfThreads;  // operand rows per thread: four threads a row
+constexpr int kWarpTma = kNumXf, kWarpMma = kNumXf + 1, kWarpPrep0 = kNumXf + 2, kNumPrep = 2;
+constexpr int kWarpEpi0 = kNumXf + 4, kNumEpi = 8;  // two epilogue warps per TMEM lane quarter
+constexpr int kWarps = kWarpEpi0 + kNumEpi;
 constexpr int kThreads = kWarps * 32;
+// registers per thread at launch: 65536 / threads, rounded down to the
+// allocation unit of 8
+constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
 // 1.5 * 2^23: its bit pattern plus an integer |s| < 2^22 is the float
 // 1.5 * 2^23 + s exactly
 constexpr uint32_t kMagicI = 0x4B400000u;
 constexpr float kMagicF = 12582912.0f;
-// registers per thread of each warpgroup (sums to 512 threads x 128
-// registers, the launch allocation)
+// registers per thread of each warpgroup; together within the launch
+// allocation
 constexpr int kRegXf = 48, kRegMisc = 96, kRegEpi = 184;
-static_assert(128 * kRegXf + 128 * kRegMisc + 256 * kRegEpi == kThreads * 128, "register pool");
+static_assert(32 * kNumXf * kRegXf + 128 * kRegMisc + 32 * kNumEpi * kRegEpi <=
+                  kThreads * kLaunchRegs,
+              "register pool");
 
 template <int BT>
 struct Cfg {
-  static constexpr int NACC = BT >= 256 ? 2 : 4;      // TMEM accumulators
-  static constexpr int CSLOTS = BT >= 256 ? 8 : 16;   // per-group constant slots
-  static constexpr int CBATCH = BT >= 128 ? 2 : 4;    // groups of constants per round trip
+  static constexpr int NACC = 4;                      // TMEM accumulators
+  static constexpr int CSLOTS = 16;                   // per-group constant slots
+  static constexpr int CBATCH = 4;                    // groups of constants per round trip
   static constexpr int COLS = BT / 2;                 // tokens per epilogue warp
-  static constexpr int CH = COLS < 16 ? COLS : 16;    // columns per TMEM load
+  static constexpr int CH = COLS < 32 ? COLS : 32;    // columns per TMEM load
 };
 
 struct Params {
@@ -117,12 +123,8 @@ __device__ __forceinline__ TileCoord tile_coord(const Params &p, int tile) {
 }
 
 __host__ __device__ constexpr int tmem_cols(int bt) {
-  // accumulators x bt, rounded up to a power of two >= 32
-  return (bt >= 256 ? 2 : 4) * bt <= 32    ? 32
-         : (bt >= 256 ? 2 : 4) * bt <= 64  ? 64
-         : (bt >= 256 ? 2 : 4) * bt <= 128 ? 128
-         : (bt >= 256 ? 2 : 4) * bt <= 256 ? 256
-                                           : 512;
+  // four accumulators of bt columns, rounded up to a power of two >= 32
+  return 4 * bt <= 32 ? 32 : 4 * bt <= 64 ? 64 : 4 * bt <= 128 ? 128 : 4 * bt <= 256 ? 256 : 512;
 }
 
 __host__ __device__ constexpr int stage_bytes(int mode, int bt) {
@@ -132,11 +134,11 @@ __host__ __device__ constexpr int stage_bytes(int mode, int bt) {
   return (BW * 128 + bt * 128 + (mode ? 2 : 1) * BW * 64 + 1023) / 1024 * 1024;
 }
 
-// one constant slot: row scales (128 fp32), per-token constants c and
-// activation scales (bt x 4 B each)
+// one constant slot: row scales (128 fp32), per-token constants c (int32)
+// and activation scales (bt x 4 B each)
 __host__ __device__ constexpr int cslot_bytes(int bt) { return BW * 4 + 2 * bt * 4; }
 
-__host__ __device__ constexpr int cslots(int bt) { return bt >= 256 ? 8 : 16; }
+__host__ __device__ constexpr int cslots(int) { return 16; }
 
 __host__ __device__ constexpr int smem_total(int mode, int bt, int stages) {
   return 1024 + stages * stage_bytes(mode, bt) + cslots(bt) * cslot_bytes(bt) +
@@ -179,8 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // constant slot c: [row scales][per-token constants][act. scales]
   uint8_t *cbase = smem + S * STAGE;
   auto sSg = [&](int c) { return reinterpret_cast<float *>(cbase + c * CSLOT); };
-  auto sCv = [&](int c) { return sSg(c) + BW; };
-  auto sXv = [&](int c) { return sCv(c) + BT; };
+  auto sCv = [&](int c) { return reinterpret_cast<int32_t *>(sSg(c) + BW); };
+  auto sXv = [&](int c) { return reinterpret_cast<float *>(sCv(c) + BT); };
   uint64_t *bars = reinterpret_cast<uint64_t *>(cbase + CS * CSLOT);
   uint64_t *fullB = bars;                      // activation and plane tiles landed
   uint64_t *fullA = bars + kMaxStages;         // byte operand written
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&stageFree[s], 1);
     }
     for (int c = 0; c < CS; ++c) {
-      mbar_init(&fullC[c], XS ? 1 + kNumXf : 1);
+      mbar_init(&fullC[c], XS ? 1 + kNumXf : 1);  // one prep warp per slot
       mbar_init(&emptyC[c], kNumEpi);
     }
     for (int b = 0; b < NACC; ++b) {
@@ -227,9 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < kWarpXf0 + kNumXf) {
     setmaxnreg_dec<kRegXf>();
     // ---------------------------------------------- plane -> operand bytes
-    // thread t: rows pass * 32 + t / 4 (pass 0..3), 16-byte plane chunk
-    // t % 4 of the group (32 columns) -> 32 operand bytes of that row
-    const int t = threadIdx.x - kWarpXf0 * 32;  // 0..127
+    // thread t: rows pass * (threads / 4) + t / 4, 16-byte plane chunk t % 4
+    // of the group (32 columns) -> 32 operand bytes of that row
+    const int t = threadIdx.x - kWarpXf0 * 32;
     const int qd = t & 3;
     int s = 0, it = 0;
     uint32_t ph = 0;  // stage slot and the parity of its current fill
@@ -243,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t *ls = sL(s);
         uint8_t *as = sA(s);
 #pragma unroll
-        for (int pass = 0; pass < 4; ++pass) {
-          const int r = pass * 32 + (t >> 2);
+        for (int pass = 0; pass < kXfPasses; ++pass) {
+          const int r = pass * (kXfThreads / 4) + (t >> 2);
           const uint4 h = *reinterpret_cast<const uint4 *>(hs + r * 64 + qd * 16);
           uint4 l = make_uint4(0, 0, 0, 0);
           if (MODE) l = *reinterpret_cast<const uint4 *>(ls + r * 64 + qd * 16);
@@ -276,17 +278,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (XS) {
           // the tokens' sums of this group from the landed activation tile
           // (rows of 128 bytes in the 128-byte swizzle): eight threads per
-          // row, one 16-byte chunk each, c = 1.5 * 2^23 + offset * sum
+          // row, one 16-byte chunk each; c = bits(1.5 * 2^23) - offset * sum
           cs = it % CS;
           ok = mbar_wait_warp(&emptyC[cs], ((it / CS) & 1) ^ 1);
           if (!ok) break;
-          float *cv = sCv(cs);
+          int32_t *cv = sCv(cs);
           const uint8_t *bs = sB(s);
           const int q = t & 7;
 #pragma unroll 4
-          for (int r0 = 0; r0 < BT; r0 += 16) {
+          for (int r0 = 0; r0 < BT; r0 += kXfThreads / 8) {
             const int r = r0 + (t >> 3);
-            const uint4 w = *reinterpret_cast<const uint4 *>(bs + r * 128 + ((q ^ (r & 7)) << 4));
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (r < BT) w = *reinterpret_cast<const uint4 *>(bs + r * 128 + ((q ^ (r & 7)) << 4));
             int sum = __dp4a((int)w.x, 0x01010101, 0);
             sum = __dp4a((int)w.y, 0x01010101, sum);
             sum = __dp4a((int)w.z, 0x01010101, sum);
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sum += __shfl_xor_sync(0xffffffffu, sum, 1);
             sum += __shfl_xor_sync(0xffffffffu, sum, 2);
             sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-            if (q == 0) cv[r] = kMagicF + (float)(OFF * sum);  // exact: |OFF * sum| < 2^22
+            if (q == 0 && r < BT) cv[r] = (int)kMagicI - OFF * sum;
           }
         }
         __syncwarp();
@@ -358,16 +361,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
         const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
         for (int g = tc.g0; g < tc.g1; ++g) {
-          // accEmpty[b] completes once per seeding of the accumulator: the
-          // epilogue seeds every accumulator once before the first group
-          ok = mbar_wait(&fullB[s], ph) && mbar_wait(&fullA[s], ph) && mbar_wait(&accEmpty[b], bph);
+          ok = mbar_wait(&fullB[s], ph) && mbar_wait(&fullA[s], ph) &&
+               mbar_wait(&accEmpty[b], bph ^ 1u);
           if (!ok) break;
           tc_fence_after();
           const uint64_t ad = ad0 + (uint64_t)s * kStageDesc, bd = bd0 + (uint64_t)s * kStageDesc;
           const uint32_t dt = tmem + (uint32_t)(b * BT);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // 4 x K=32 bytes inside the 128-byte row
-            umma_i8(dt, ad + 2 * kk, bd + 2 * kk, IDESC, 1u);  // onto the seed
+            umma_i8(dt, ad + 2 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
           umma_commit(&stageFree[s]);
           umma_commit(&accFull[b]);
           issued = true;
@@ -387,20 +389,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // after a wait gave up): commits complete in order
       if (issued) mbar_wait_final(&accFull[lb], lbph);
     }
-    } else if (warp == kWarpPrep) {
+    } else if (warp >= kWarpPrep0) {
     // ----------------------------------------------- per-group constants
     // CBATCH groups per round trip: lane i holds rows i + 32 r (r < 4) and
     // tokens i + 32 u (u < BT / 32, at least one), all loads of a batch
-    // issued before the first use.
+    // issued before the first use.  Two warps take turns batch by batch, so
+    // two round trips are in flight.
     constexpr int TU = BT < 32 ? 1 : BT / 32;
     constexpr int CB = C::CBATCH;
+    const int pw = warp - kWarpPrep0;
     griddep_wait();
-    int it = 0;
+    int it = 0, batch = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
       const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
       const int n0 = tc.n0, m0 = tc.m0, G1 = tc.g1, G = p.G;
-      for (int gb = tc.g0; gb < G1 && ok; gb += CB) {
+      for (int gb = tc.g0; gb < G1 && ok; gb += CB, ++batch) {
+        if (batch % kNumPrep != pw) {  // the other warp's batch
+          it += min(CB, G1 - gb);
+          continue;
+        }
         uint16_t sv[4][CB];
         int rv[TU][CB];
         float xv[TU][CB];
@@ -430,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait_warp(&emptyC[c], ((it / CS) & 1) ^ 1);
           if (!ok) break;
           float *sg = sSg(c);
-          float *cv = sCv(c);
+          int32_t *cv = sCv(c);
           float *xs = sXv(c);
 #pragma unroll
           for (int r = 0; r < 4; ++r) sg[lane + 32 * r] = __half2float(__ushort_as_half(sv[r][k]));
@@ -438,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < TU; ++u) {
             const int j = lane + 32 * u;
             if (j < BT) {
-              if (!XS) cv[j] = kMagicF + (float)(OFF * rv[u][k]);  // exact
+              if (!XS) cv[j] = (int)kMagicI - OFF * rv[u][k];
               if (ACTG) xs[j] = xv[u][k];
             }
           }
@@ -458,16 +466,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;
     const int col0 = half * COLS;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    // seed every accumulator before its first group
-#pragma unroll
-    for (int b = 0; b < NACC; ++b)
-#pragma unroll
-      for (int c = 0; c < COLS; c += CH) tmem_st_const<CH>(tmem + lane_addr + b * BT + col0 + c, kMagicI);
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0)
-      for (int b = 0; b < NACC; ++b) mbar_arrive(&accEmpty[b]);
     griddep_wait();  // y may still be read by the preceding kernel
     int it = 0;
     bool ok = true;
@@ -485,32 +483,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) continue;
         tc_fence_after();
         const float sg = sSg(cs)[row];
-        const float *cv = sCv(cs) + col0;
+        const int32_t *cv = sCv(cs) + col0;
         const float *xv = sXv(cs) + col0;
+        // the whole group is read out and the accumulator handed back to the
+        // MMA before the arithmetic
+        const uint32_t ta0 = tmem + lane_addr + b * BT + col0;
+        uint32_t dd[COLS];
+#pragma unroll
+        for (int c = 0; c < COLS; c += CH)
+          tmem_ld<CH>(ta0 + c, *reinterpret_cast<uint32_t(*)[CH]>(dd + c));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accEmpty[b]);
 #pragma unroll
         for (int c = 0; c < COLS; c += CH) {
-          const uint32_t ta = tmem + lane_addr + b * BT + col0 + c;
-          uint32_t d[CH];
-          tmem_ld<CH>(ta, d);
-          tmem_ld_wait();
-          tmem_st_const<CH>(ta, kMagicI);  // seed for the accumulator's next group
+          const uint32_t *d = dd + c;
           if (DEBUG) {
 #pragma unroll
             for (int j = 0; j < CH; ++j) {
               const int m = m0 + col0 + c + j;
-              if (m < p.M && n < p.N)  // exact: both are integers of one binade
-                p.S[((int64_t)m * p.N + n) * p.G + g] =
-                    __float2int_rn(__int_as_float((int)d[j]) - cv[c + j]);
+              if (m < p.M && n < p.N)
+                p.S[((int64_t)m * p.N + n) * p.G + g] = (int)d[j] + cv[c + j] - (int)kMagicI;
             }
           } else {
 #pragma unroll
             for (int j = 0; j < CH; j += 4) {
-              const float4 c4 = *reinterpret_cast<const float4 *>(cv + c + j);
-              // 1.5 * 2^23 + raw sum, minus 1.5 * 2^23 + offset * sum(q): exact
-              float f0 = __int_as_float((int)d[j]), f1 = __int_as_float((int)d[j + 1]);
-              float f2 = __int_as_float((int)d[j + 2]), f3 = __int_as_float((int)d[j + 3]);
-              f32x2_sub(f0, f1, f0, f1, c4.x, c4.y);
-              f32x2_sub(f2, f3, f2, f3, c4.z, c4.w);
+              const int4 c4 = *reinterpret_cast<const int4 *>(cv + c + j);
+              // 1.5 * 2^23 + exact group sum, as a float, minus the magic
+              float f0 = __int_as_float((int)d[j] + c4.x), f1 = __int_as_float((int)d[j + 1] + c4.y);
+              float f2 = __int_as_float((int)d[j + 2] + c4.z), f3 = __int_as_float((int)d[j + 3] + c4.w);
+              f32x2_add(f0, f1, f0, f1, -kMagicF, -kMagicF);
+              f32x2_add(f2, f3, f2, f3, -kMagicF, -kMagicF);
               float s0 = sg, s1 = sg, s2 = sg, s3 = sg;
               if (ACTG) {
                 const float4 x4 = *reinterpret_cast<const float4 *>(xv + c + j);
@@ -524,13 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        tmem_st_wait();
-        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&accEmpty[b]);
-          mbar_arrive(&emptyC[cs]);
-        }
+        if (lane == 0) mbar_arrive(&emptyC[cs]);
       }
       if constexpr (SPLIT && !DEBUG) {
         // this range's partial sums of the warp's sub-block (rows of its lane
@@ -620,14 +619,12 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
-// Token tile: 256 from 512 tokens up (each transformed weight tile serves
-// twice the tokens; prefill), else the smallest of 16 .. 128 that holds M.
+// Token tile: the smallest of 16 .. 128 that holds M (128 from there on).
 int pick_bt(int64_t M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
-  if (M < 512) return 128;
-  return 256;
+  return 128;
 }
 
 int pick_stages(int mode, int bt, int max_smem) {
@@ -652,7 +649,6 @@ int num_sms() {
 // per epilogue warp and tile) at a fixed place, the start, so that calls of
 // any shapes can share one scratch (each leaves its counters zero, and no
 // shape's partial tiles reach another's counters); then the partial tiles.
-// Tiles of 256 tokens are never split.
 constexpr int kMaxCntTiles = 256;
 constexpr int64_t kCntBytes = int64_t(kMaxCntTiles) * kNumEpi * 4;  // 8 KB
 struct SplitPlan {
@@ -665,7 +661,7 @@ SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int bt) {
   sp.tmn = ((N + BW - 1) / BW) * ((M + bt - 1) / bt);
   const int sms = num_sms();
   int s = 1;
-  if (bt <= 128 && sp.tmn * 2 <= sms && sp.tmn <= kMaxCntTiles) {
+  if (sp.tmn * 2 <= sms && sp.tmn <= kMaxCntTiles) {
     s = (int)(sms / sp.tmn);
     if (s > G / 4) s = G / 4;
     if (s < 1) s = 1;
@@ -676,7 +672,7 @@ SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int bt) {
   return sp;
 }
 
-// The register split hands out exactly the launch allocation of 128
+// The register split hands out the launch allocation of kLaunchRegs
 // registers per thread; a kernel built with fewer would make the increase
 // wait for registers that do not exist, so it is not launched.
 template <typename Kern>
@@ -684,7 +680,7 @@ cudaError_t check_register_pool(Kern kern) {
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
-  return fa.numRegs == 128 ? cudaSuccess : cudaErrorInvalidConfiguration;
+  return fa.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
 }
 
 template <int MODE, int BT, bool ACTG, bool DEBUG, bool XS>
@@ -737,7 +733,7 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   p.stages = stages;
   const int grid = p.tiles < num_sms() ? p.tiles : num_sms();
   const int smem = smem_total(MODE, BT, stages);
-  constexpr bool kCanSplit = !DEBUG && BT <= 128;
+  constexpr bool kCanSplit = !DEBUG;
   auto kern = (kCanSplit && p.splits > 1) ? tc_linear_kernel<MODE, BT, ACTG, DEBUG, kCanSplit, XS>
                                           : tc_linear_kernel<MODE, BT, ACTG, DEBUG, false, XS>;
   cudaError_t e = check_register_pool(kern);
@@ -769,8 +765,7 @@ cudaError_t launch_mode(const LinearArgs &a, cudaStream_t st) {
     case 16: return launch_g<MODE, 16, DEBUG>(a, st);
     case 32: return launch_g<MODE, 32, DEBUG>(a, st);
     case 64: return launch_g<MODE, 64, DEBUG>(a, st);
-    case 128: return launch_g<MODE, 128, DEBUG>(a, st);
-    default: return launch_g<MODE, 256, DEBUG>(a, st);
+    default: return launch_g<MODE, 128, DEBUG>(a, st);
   }
 }
 
