@@ -783,6 +783,72 @@ def measure_round(wl, hbm_peak, reps=10):
     }
 
 
+# ------------------------------------------ speculative decoding rounds
+SPEC_DIM, SPEC_LAYERS, SPEC_VOCAB, SPEC_GAMMA = 4096, 4, 8192, 3
+
+
+def measure_speculative(wl, hbm_peak, replays=40):
+    """Speculative rounds (gamma = 3) against the target's own greedy
+    decoding on a synthetic nested model (dim 4096, 4 layers, vocabulary
+    8192; planes and scales packed by bitnest_pack_weights from seeded
+    N(0, 0.02^2) fp16 weights, so the draft is close to the target).  One
+    round and one greedy step are each captured as a CUDA graph (the
+    sequence and its length stay on the device) and replayed; CUDA events."""
+    import torch
+
+    bn = wl.bn
+    dev = wl.dev
+    d, L, V, gamma = SPEC_DIM, SPEC_LAYERS, SPEC_VOCAB, SPEC_GAMMA
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(synth.SEED_WEIGHTS + 900)
+
+    def packed(rows):
+        w = (0.02 * torch.randn((rows, d), generator=gen, device=dev)).half()
+        return bn.pack_weights(w)
+
+    model = bn.SpecModel(torch.randn((V, d), generator=gen, device=dev).half(),
+                         [packed(d) for _ in range(L)], packed(V))
+    cap = 2 + (replays + 4) * (gamma + 1)
+
+    def state(g):
+        seq = torch.zeros((cap,), dtype=torch.int32, device=dev)
+        seq[:2] = torch.tensor([1, 2], dtype=torch.int32)
+        return (seq, torch.tensor([2], dtype=torch.int32, device=dev),
+                torch.zeros(4, dtype=torch.int32, device=dev),
+                torch.empty(bn.spec_work_bytes(V, d, g), dtype=torch.uint8, device=dev))
+
+    res = {}
+    for name, g, fn in (("speculative", gamma, lambda st: bn.spec_rounds(model, gamma, 1, *st)),
+                        ("target_greedy", 0, lambda st: bn.spec_greedy(model, 1, *st))):
+        st = state(g)
+        graph = capture(lambda: fn(st))  # one round (or step) already ran while warming
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        st[2].zero_()
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(replays):
+            graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        t = a.elapsed_time(b) / 1e3
+        rounds, appended, accepted, overflow = (int(v) for v in st[2].tolist())
+        graph.reset()
+        res[name] = {"us_per_call": round(t / replays * 1e6, 2),
+                     "tokens_per_s": round(appended / t, 1),
+                     "tokens_per_call": round(appended / replays, 3)}
+        if g:
+            res[name]["acceptance"] = round(accepted / max(1, rounds * gamma), 4)
+        if overflow:
+            res[name]["error"] = "sequence capacity exceeded"
+    res["speedup_vs_target_greedy"] = round(res["speculative"]["tokens_per_s"] /
+                                            res["target_greedy"]["tokens_per_s"], 3)
+    del model
+    return {"workload": f"synthetic nested model: dim {d}, {L} layers, vocabulary {V}, "
+                        f"gamma {gamma}; one round / one greedy step per CUDA graph replay",
+            **res}
+
+
 # ------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -799,7 +865,7 @@ def main():
                          "(for profilers that cannot replay the captured kernel nodes)")
     ap.add_argument("--workload", default="all",
                     choices=["all", "decode", "prefill", "sweep", "round", "pack", "hadamard",
-                             "attention"],
+                             "attention", "spec"],
                     help="all: the decode step line with the prefill, M-sweep and "
                          "decode-round objects; otherwise only that part (profiling runs)")
     args = ap.parse_args()
@@ -862,6 +928,12 @@ def main():
             "per_projection": pre,
             "l2": "flushed (256 MB write) before every timed launch",
         }
+    spec_res = None
+    if args.workload in ("all", "spec"):
+        try:
+            spec_res = measure_speculative(wl, hbm_peak)
+        except Exception as e:  # noqa: BLE001
+            spec_res = {"error": f"{type(e).__name__}: {e}"}
     att = None
     if args.workload in ("all", "attention"):
         # an auxiliary row, measured last: its failure must not cost the rest
@@ -875,7 +947,7 @@ def main():
         if rank == 0:
             part = {"prefill": prefill, "m_sweep": sweep, "decode_round": rnd,
                     "pack_from_weights": pack, "down_proj_input_rotation": had,
-                    "nested_kv_attention": att}
+                    "nested_kv_attention": att, "speculative_rounds": spec_res}
             print(json.dumps({"metric": METRIC, "workload": f"{args.workload} only",
                               **{k: v for k, v in part.items() if v is not None}}), flush=True)
         return
@@ -918,6 +990,8 @@ def main():
         out["down_proj_input_rotation"] = had
     if att is not None:
         out["nested_kv_attention"] = att
+    if spec_res is not None:
+        out["speculative_rounds"] = spec_res
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, cores, rows = cpu_baseline()
         out["cpu_baseline"] = {

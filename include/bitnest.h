@@ -316,6 +316,65 @@ int bitnest_quantize_linear(int mode, const uint8_t *hi, const uint8_t *lo,
                             int64_t K, float *y, int act_group, const uint16_t *bias,
                             int8_t *xq, float *xscale, int32_t *xsum, int path, void *stream);
 
+/*
+ * Speculative decoding with the nested weights (BitNest-Llama-3-8B model
+ * card, opening paragraph: the W4A8 draft proposes tokens and the W8A8
+ * target verifies every one of them, so the output is exactly the target's
+ * greedy output; model table row "Default draft length": gamma = 3).  The
+ * pages give no model; these entry points run a small synthetic one built
+ * from the nested linear layer (bitnest_quantize_linear per layer):
+ *   input at position p : x0 = fp16(E[t_p] + 0.5 E[t_{p-1}])   (t_{-1} := t_0)
+ *   layer l             : x_{l+1} = fp16(tanh(W_l x_l)),  W_l nested [dim, dim]
+ *   head                : logits = W_head x_L,             W_head nested [vocab, dim]
+ *   next token          : argmax of the logits, lowest index among equal maxima
+ * A round: gamma draft steps (draft weights, one token each), one target pass
+ * over the gamma + 1 positions together, then the accept step appends the
+ * leading draft tokens the target agrees with and the target's own token
+ * after them (1 .. gamma + 1 tokens).  The sequence, its length and the
+ * statistics live in device memory: nothing is read back to the host, and
+ * the rounds can be captured in a CUDA graph.
+ *   model  : host struct; embed fp16 [vocab, dim]; hi / lo / scale are HOST
+ *            arrays of `layers` DEVICE pointers (planes uint8 [dim, dim/2],
+ *            scales fp16 [dim, dim/128]); head planes [vocab, dim/2], scales
+ *            [vocab, dim/128].  dim a positive multiple of 128.
+ *   seq    : int32 [cap] device, tokens 0 .. *len - 1 on entry (*len >= 1);
+ *            tokens are appended.  The caller keeps cap >= *len + rounds *
+ *            (gamma + 1) (greedy: + steps); a write that would pass cap is
+ *            not made and sets stats[3].
+ *   len    : int32 device scalar, updated in place.
+ *   stats  : int32 [4] device, accumulated: rounds, tokens appended, draft
+ *            tokens accepted, capacity overflow flag.
+ *   work   : device scratch of bitnest_spec_work_bytes(vocab, dim, gamma)
+ *            bytes (16-byte aligned), owned by the caller.
+ * gamma in 0 .. BITNEST_GEMV_MAX_M - 1.  Checks and errors as the other
+ * entry points; everything is asynchronous on `stream`.
+ */
+typedef struct bitnest_spec_model {
+  int64_t vocab, dim, layers;
+  const uint16_t *embed;
+  const uint8_t *const *hi;
+  const uint8_t *const *lo;
+  const uint16_t *const *scale;
+  const uint8_t *head_hi;
+  const uint8_t *head_lo;
+  const uint16_t *head_scale;
+} bitnest_spec_model;
+
+/* Scratch bytes of a round (or of greedy decoding with gamma = 0);
+ * -BITNEST_ERR_UNSUPPORTED_SHAPE for a bad shape.  Host only. */
+int64_t bitnest_spec_work_bytes(int64_t vocab, int64_t dim, int gamma);
+
+/* `rounds` speculative rounds with draft length `gamma`. */
+int bitnest_spec_rounds(const bitnest_spec_model *model, int gamma, int rounds, int32_t *seq,
+                        int64_t cap, int32_t *len, int32_t *stats, void *work,
+                        int64_t work_bytes, void *stream);
+
+/* `steps` tokens of the target's own greedy decoding (one position per step):
+ * the sequence speculative rounds must reproduce. */
+int bitnest_spec_greedy(const bitnest_spec_model *model, int steps, int32_t *seq, int64_t cap,
+                        int32_t *len, int32_t *stats, void *work, int64_t work_bytes,
+                        void *stream);
+
 /* The kernel family BITNEST_PATH_AUTO picks for this problem (host only,
  * launches nothing).  Returns BITNEST_PATH_GEMV or BITNEST_PATH_TC. */
 int bitnest_select_path(int mode, int64_t M, int64_t N, int64_t K);

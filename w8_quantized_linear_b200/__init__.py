@@ -69,12 +69,16 @@ def lib() -> ctypes.CDLL:
     L.bitnest_linear_static_ws.argtypes = [I, P, P, P, P, P, P, I64, I64, I64, P, I, P, I, P]
     L.bitnest_linear_ws_bytes.argtypes = [I, I64, I64, I64, I]
     L.bitnest_linear_ws_bytes.restype = I64
+    L.bitnest_spec_work_bytes.argtypes = [I64, I64, I]
+    L.bitnest_spec_work_bytes.restype = I64
+    L.bitnest_spec_rounds.argtypes = [P, I, I, P, I64, P, P, P, I64, P]
+    L.bitnest_spec_greedy.argtypes = [P, I, P, I64, P, P, P, I64, P]
     for name in ("bitnest_pack_planes", "bitnest_pack_weights", "bitnest_quantize_act",
                  "bitnest_act_group_sums", "bitnest_hadamard_quantize_act",
                  "bitnest_nested_attention",
                  "bitnest_linear", "bitnest_linear_path", "bitnest_select_path",
                  "bitnest_debug_group_sums", "bitnest_quantize_linear", "bitnest_linear_ws",
-                 "bitnest_linear_static_ws"):
+                 "bitnest_linear_static_ws", "bitnest_spec_rounds", "bitnest_spec_greedy"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -305,3 +309,53 @@ def debug_group_sums(mode: int, hi, lo, xq, xsum, path: int = PATH_AUTO, out=Non
                                           M, N, K, _ptr(S), int(path), _stream(xq)),
            "bitnest_debug_group_sums")
     return S
+
+
+# ------------------------------------------------- speculative decoding
+class _SpecModelC(ctypes.Structure):
+    _fields_ = [("vocab", ctypes.c_int64), ("dim", ctypes.c_int64), ("layers", ctypes.c_int64),
+                ("embed", ctypes.c_void_p), ("hi", ctypes.POINTER(ctypes.c_void_p)),
+                ("lo", ctypes.POINTER(ctypes.c_void_p)),
+                ("scale", ctypes.POINTER(ctypes.c_void_p)), ("head_hi", ctypes.c_void_p),
+                ("head_lo", ctypes.c_void_p), ("head_scale", ctypes.c_void_p)]
+
+
+class SpecModel:
+    """The synthetic model of bitnest_spec_rounds: embed fp16 [V, d] and
+    (hi, lo, scale) device tensors per layer ([d, d/2] planes, [d, d/128]
+    scales) and for the head ([V, d/2], [V, d/128]).  Holds the C struct."""
+
+    def __init__(self, embed, layers, head):
+        self.embed, self.layers, self.head = embed, list(layers), head
+        self.vocab, self.dim = embed.shape
+        n = len(self.layers)
+        self._hi = (ctypes.c_void_p * max(n, 1))(*[t[0].data_ptr() for t in self.layers])
+        self._lo = (ctypes.c_void_p * max(n, 1))(*[t[1].data_ptr() for t in self.layers])
+        self._sc = (ctypes.c_void_p * max(n, 1))(*[t[2].data_ptr() for t in self.layers])
+        self.c = _SpecModelC(self.vocab, self.dim, n, embed.data_ptr(),
+                             ctypes.cast(self._hi, ctypes.POINTER(ctypes.c_void_p)),
+                             ctypes.cast(self._lo, ctypes.POINTER(ctypes.c_void_p)),
+                             ctypes.cast(self._sc, ctypes.POINTER(ctypes.c_void_p)),
+                             head[0].data_ptr(), head[1].data_ptr(), head[2].data_ptr())
+
+
+def spec_work_bytes(vocab: int, dim: int, gamma: int) -> int:
+    n = lib().bitnest_spec_work_bytes(int(vocab), int(dim), int(gamma))
+    if n < 0:
+        _check(-n, "bitnest_spec_work_bytes")
+    return n
+
+
+def spec_rounds(model: SpecModel, gamma: int, rounds: int, seq, length, stats, work):
+    """`rounds` speculative rounds on the device sequence `seq` (int32 [cap]),
+    `length` (int32 [1]) and `stats` (int32 [4]), scratch `work` (uint8)."""
+    _check(lib().bitnest_spec_rounds(ctypes.byref(model.c), int(gamma), int(rounds), _ptr(seq),
+                                     seq.numel(), _ptr(length), _ptr(stats), _ptr(work),
+                                     work.numel(), _stream(seq)), "bitnest_spec_rounds")
+
+
+def spec_greedy(model: SpecModel, steps: int, seq, length, stats, work):
+    """`steps` tokens of the target's greedy decoding, same buffers."""
+    _check(lib().bitnest_spec_greedy(ctypes.byref(model.c), int(steps), _ptr(seq), seq.numel(),
+                                     _ptr(length), _ptr(stats), _ptr(work), work.numel(),
+                                     _stream(seq)), "bitnest_spec_greedy")
