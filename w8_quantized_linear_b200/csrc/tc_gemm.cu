@@ -12,8 +12,17 @@
 // up to 128), one 128-column group per pipeline stage.  The group scales
 // differ per (row, group), so the int32 accumulator of every group is
 // drained from TMEM and scaled in fp32 (the model card's per-group scale);
-// four TMEM accumulators let the drain of a group run while the MMAs of the
-// next three proceed.
+// three TMEM accumulators let the drain of a group run while the MMAs of the
+// next two proceed.
+//
+// The weight operand never touches shared memory: each thread of the
+// transform warps owns one weight row, reads its plane bytes of the group
+// from a 64-byte-swizzled TMA tile (conflict-free, one row per lane) and
+// writes the 128 operand bytes into a TMEM slot of the stage, from which the
+// MMA reads A.  Shared memory then carries only the activation tile (the
+// MMA's B), the plane tiles and the per-group constants: the operand's store
+// and the MMA's reads of it were the bulk of the shared-memory traffic that
+// bounded this kernel.
 //
 // The drain turns each int32 group sum into fp32 exactly with one integer
 // add: the bit pattern of 1.5 * 2^23 minus offset * sum(q) (one constant per
@@ -29,9 +38,9 @@
 // next tile while the epilogue finishes the current one.
 //
 // Warp roles (16 warps, four warpgroups):
-//   0..3   plane -> byte operand (shared-memory planes -> swizzled K-major);
-//          without caller group sums also the tokens' sums of the group
-//          (from the landed activation tile)
+//   0..3   plane -> byte operand (shared-memory planes -> TMEM, one row per
+//          thread); without caller group sums also the tokens' sums of the
+//          group (from the landed activation tile)
 //   4      TMA producer: activation tile (128-byte swizzle) and the hi / lo
 //          plane tiles of the group, one mbarrier per stage (this CTA only)
 //   5      TMEM owner and MMA issuer (one thread)
@@ -58,7 +67,6 @@ constexpr int BW = 128;  // weight rows per tile
 constexpr int kMaxStages = 8;
 constexpr int kWarpXf0 = 0, kNumXf = 4;  // one warpgroup
 constexpr int kXfThreads = 32 * kNumXf;
-constexpr int kXfPasses = 4 * 128 / kXfThreads;  // operand rows per thread: four threads a row
 constexpr int kWarpTma = kNumXf, kWarpMma = kNumXf + 1, kWarpPrep0 = kNumXf + 2, kNumPrep = 2;
 constexpr int kWarpEpi0 = kNumXf + 4, kNumEpi = 8;  // two epilogue warps per TMEM lane quarter
 constexpr int kWarps = kWarpEpi0 + kNumEpi;
@@ -72,14 +80,14 @@ constexpr uint32_t kMagicI = 0x4B400000u;
 constexpr float kMagicF = 12582912.0f;
 // registers per thread of each warpgroup; together within the launch
 // allocation
-constexpr int kRegXf = 48, kRegMisc = 96, kRegEpi = 184;
+constexpr int kRegXf = 56, kRegMisc = 96, kRegEpi = 176;
 static_assert(32 * kNumXf * kRegXf + 128 * kRegMisc + 32 * kNumEpi * kRegEpi <=
                   kThreads * kLaunchRegs,
               "register pool");
 
 template <int BT>
 struct Cfg {
-  static constexpr int NACC = 4;                      // TMEM accumulators
+  static constexpr int NACC = 3;                      // TMEM accumulators
   static constexpr int CSLOTS = 16;                   // per-group constant slots
   static constexpr int CBATCH = 4;                    // groups of constants per round trip
   static constexpr int COLS = BT / 2;                 // tokens per epilogue warp
@@ -122,16 +130,19 @@ __device__ __forceinline__ TileCoord tile_coord(const Params &p, int tile) {
   return c;
 }
 
+// Tensor memory: three accumulators of bt columns, then one 32-column slot
+// of the weight operand per pipeline stage (128 bytes of K per lane).
+constexpr int kStagesMax = 4;
+__host__ __device__ constexpr int tmem_abase(int bt) { return (3 * bt + 31) / 32 * 32; }
 __host__ __device__ constexpr int tmem_cols(int bt) {
-  // four accumulators of bt columns, rounded up to a power of two >= 32
-  return 4 * bt <= 32 ? 32 : 4 * bt <= 64 ? 64 : 4 * bt <= 128 ? 128 : 4 * bt <= 256 ? 256 : 512;
+  // rounded up to a power of two >= 32
+  return tmem_abase(bt) + 32 * kStagesMax <= 256 ? 256 : 512;
 }
 
 __host__ __device__ constexpr int stage_bytes(int mode, int bt) {
-  // operand A (128 x 128 B), operand B (bt x 128 B), hi (and lo) plane tiles
-  // (128 x 64 B each); stages start on 1024-byte boundaries (the 128-byte
-  // swizzle atom)
-  return (BW * 128 + bt * 128 + (mode ? 2 : 1) * BW * 64 + 1023) / 1024 * 1024;
+  // operand B (bt x 128 B, 128-byte swizzle), hi (and lo) plane tiles
+  // (128 x 64 B each, 64-byte swizzle); stages start on 1024-byte boundaries
+  return (bt * 128 + (mode ? 2 : 1) * BW * 64 + 1023) / 1024 * 1024;
 }
 
 // one constant slot: row scales (128 fp32), per-token constants c (int32)
@@ -173,11 +184,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   const int S = p.stages;
-  // stage s: [A 16 KB][B bt x 128][hi 8 KB][lo 8 KB]
-  auto sA = [&](int s) { return smem + s * STAGE; };
-  auto sB = [&](int s) { return smem + s * STAGE + BW * 128; };
-  auto sH = [&](int s) { return smem + s * STAGE + BW * 128 + BT * 128; };
-  auto sL = [&](int s) { return smem + s * STAGE + BW * 128 + BT * 128 + BW * 64; };
+  // stage s: [B bt x 128][hi 8 KB][lo 8 KB]; its weight operand is in tensor
+  // memory (slot s)
+  auto sB = [&](int s) { return smem + s * STAGE; };
+  auto sH = [&](int s) { return smem + s * STAGE + BT * 128; };
+  auto sL = [&](int s) { return smem + s * STAGE + BT * 128 + BW * 64; };
   // constant slot c: [row scales][per-token constants][act. scales]
   uint8_t *cbase = smem + S * STAGE;
   auto sSg = [&](int c) { return reinterpret_cast<float *>(cbase + c * CSLOT); };
@@ -229,10 +240,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < kWarpXf0 + kNumXf) {
     setmaxnreg_dec<kRegXf>();
     // ---------------------------------------------- plane -> operand bytes
-    // thread t: rows pass * (threads / 4) + t / 4, 16-byte plane chunk t % 4
-    // of the group (32 columns) -> 32 operand bytes of that row
+    // thread t: weight row t of the tile (TMEM lane t, in this warp's lane
+    // quarter): its 64 hi (and lo) plane bytes of the group -> 128 operand
+    // bytes, written to the stage's TMEM slot as 32 columns
     const int t = threadIdx.x - kWarpXf0 * 32;
-    const int qd = t & 3;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int sw = (t >> 1) & 3;  // the plane tiles' 64-byte swizzle: chunk c sits at c ^ sw
     int s = 0, it = 0;
     uint32_t ph = 0;  // stage slot and the parity of its current fill
     bool ok = true;
@@ -241,39 +254,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = tc.g0; g < tc.g1; ++g, ++it) {
         ok = mbar_wait_warp(&fullB[s], ph);
         if (!ok) break;
-        const uint8_t *hs = sH(s);
-        const uint8_t *ls = sL(s);
-        uint8_t *as = sA(s);
+        const uint8_t *hs = sH(s) + t * 64;
+        const uint8_t *ls = sL(s) + t * 64;
+        const uint32_t at = tmem + lane_base + (uint32_t)(tmem_abase(BT) + 32 * s);
 #pragma unroll
-        for (int pass = 0; pass < kXfPasses; ++pass) {
-          const int r = pass * (kXfThreads / 4) + (t >> 2);
-          const uint4 h = *reinterpret_cast<const uint4 *>(hs + r * 64 + qd * 16);
-          uint4 l = make_uint4(0, 0, 0, 0);
-          if (MODE) l = *reinterpret_cast<const uint4 *>(ls + r * 64 + qd * 16);
-          const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
-          const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
-          uint32_t out[8];
+        for (int half = 0; half < 2; ++half) {  // columns 64 half .. 64 half + 63
+          uint32_t out[16];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t ev, od;  // bytes of columns 8w + {0,2,4,6} and 8w + {1,3,5,7}
-            if (MODE == 0) {
-              ev = hw[w] & 0x0F0F0F0Fu;
-              od = (hw[w] >> 4) & 0x0F0F0F0Fu;
-            } else {
-              ev = ((hw[w] << 4) & 0xF0F0F0F0u) | (lw[w] & 0x0F0F0F0Fu);
-              od = (hw[w] & 0xF0F0F0F0u) | ((lw[w] >> 4) & 0x0F0F0F0Fu);
+          for (int cc = 0; cc < 2; ++cc) {  // plane chunk c = 2 half + cc: 32 columns
+            const int c = 2 * half + cc;
+            const uint4 h = *reinterpret_cast<const uint4 *>(hs + ((c ^ sw) << 4));
+            uint4 l = make_uint4(0, 0, 0, 0);
+            if (MODE) l = *reinterpret_cast<const uint4 *>(ls + ((c ^ sw) << 4));
+            const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+            const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              uint32_t ev, od;  // bytes of columns 8w + {0,2,4,6} and 8w + {1,3,5,7}
+              if (MODE == 0) {
+                ev = hw[w] & 0x0F0F0F0Fu;
+                od = (hw[w] >> 4) & 0x0F0F0F0Fu;
+              } else {
+                ev = ((hw[w] << 4) & 0xF0F0F0F0u) | (lw[w] & 0x0F0F0F0Fu);
+                od = (hw[w] & 0xF0F0F0F0u) | ((lw[w] >> 4) & 0x0F0F0F0Fu);
+              }
+              out[8 * cc + 2 * w] = prmt(ev, od, 0x5140);      // columns 8w + 0..3
+              out[8 * cc + 2 * w + 1] = prmt(ev, od, 0x7362);  // columns 8w + 4..7
             }
-            out[2 * w] = prmt(ev, od, 0x5140);      // columns 8w + 0..3
-            out[2 * w + 1] = prmt(ev, od, 0x7362);  // columns 8w + 4..7
           }
-          // 16-byte chunks 2qd and 2qd+1 of the 128-byte row, 128-byte swizzle
-          const int c0 = 2 * qd, c1 = 2 * qd + 1;
-          *reinterpret_cast<uint4 *>(as + r * 128 + ((c0 ^ (r & 7)) << 4)) =
-              make_uint4(out[0], out[1], out[2], out[3]);
-          *reinterpret_cast<uint4 *>(as + r * 128 + ((c1 ^ (r & 7)) << 4)) =
-              make_uint4(out[4], out[5], out[6], out[7]);
+          tmem_st16(at + 16 * half, out);
         }
-        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
         int cs = 0;
         if constexpr (XS) {
           // the tokens' sums of this group from the landed activation tile
@@ -355,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0, b = 0, lb = 0;
       uint32_t ph = 0, bph = 0, lbph = 0;
       bool issued = false;
-      const uint64_t ad0 = umma_desc_sw128(sA(0)), bd0 = umma_desc_sw128(sB(0));
+      const uint64_t bd0 = umma_desc_sw128(sB(0));
+      const uint32_t at0 = tmem + (uint32_t)tmem_abase(BT);  // the weight operand slots
       constexpr uint64_t kStageDesc = STAGE >> 4;  // descriptor address unit: 16 bytes
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
@@ -365,11 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                mbar_wait(&accEmpty[b], bph ^ 1u);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t ad = ad0 + (uint64_t)s * kStageDesc, bd = bd0 + (uint64_t)s * kStageDesc;
+          const uint64_t bd = bd0 + (uint64_t)s * kStageDesc;
+          const uint32_t at = at0 + (uint32_t)(32 * s);
           const uint32_t dt = tmem + (uint32_t)(b * BT);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // 4 x K=32 bytes inside the 128-byte row
-            umma_i8(dt, ad + 2 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)  // 4 x K=32: 8 TMEM columns of A, 32 bytes of B
+            umma_i8_ta(dt, at + 8 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
           umma_commit(&stageFree[s]);
           umma_commit(&accFull[b]);
           issued = true;
@@ -628,7 +642,7 @@ int pick_bt(int64_t M) {
 }
 
 int pick_stages(int mode, int bt, int max_smem) {
-  for (int s = kMaxStages; s >= 2; --s)
+  for (int s = kStagesMax; s >= 2; --s)
     if (smem_total(mode, bt, s) <= max_smem) return s;
   return 0;
 }
@@ -692,11 +706,11 @@ cudaError_t launch_t(const LinearArgs &a, cudaStream_t st) {
   if (stages == 0) return cudaErrorInvalidValue;
   CUtensorMap mq, mh, ml;
   if (!make_map(&mq, a.xq, (uint64_t)a.M, (uint64_t)a.K, BT, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mh, a.hi, (uint64_t)a.N, (uint64_t)(a.K / 2), BW, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+      !make_map(&mh, a.hi, (uint64_t)a.N, (uint64_t)(a.K / 2), BW, 64, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   if (MODE) {
     if (!make_map(&ml, a.lo, (uint64_t)a.N, (uint64_t)(a.K / 2), BW, 64,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
+                  CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   } else {
     ml = mh;
