@@ -171,6 +171,27 @@ def group_shape(members):
     return N, K, g
 
 
+def step_host_inputs():
+    """The decode step's seeded inputs on the host: per layer group its
+    stacked nibble planes and scales, per (group, pass) its fp16 activations.
+    Only the input generators; no arithmetic of the layer."""
+    groups, acts = {}, {}
+    for gi, (gname, members) in enumerate(LAYER_GROUPS):
+        parts = []
+        for m in members:
+            N, K, _ = synth.LLAMA3_8B_PROJECTIONS[m]
+            pid = synth.PROJ_IDS[m]
+            parts.append((synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K),
+                          synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K),
+                          synth.group_scales(synth.SEED_SCALES + pid, N, K)))
+        groups[gname] = tuple(np.concatenate([p[i] for p in parts], axis=0) if len(parts) > 1
+                              else parts[0][i] for i in range(3))
+        N, K, g = group_shape(members)
+        for mode, M in DECODE_M.items():
+            acts[gname, mode] = synth.activations(synth.SEED_ACTS + 10 * gi + 100 * mode, M, K)
+    return groups, acts
+
+
 def decode_step_bytes():
     """Algorithmic bytes of one decode step (both passes, all layer groups)."""
     tot = 0
@@ -206,10 +227,10 @@ class DecodeWorkload:
             return hi, lo, torch.from_numpy(s).to(device)
 
         self.single = {name: planes(*nib[name]) for name, _ in self.projs}
-        base = {}
-        for gname, members in LAYER_GROUPS:
-            base[gname] = planes(*(np.concatenate([nib[m][i] for m in members], axis=0)
-                                   for i in range(3)))
+        del nib
+        host_groups, host_acts = step_host_inputs()
+        base = {gname: planes(*host_groups[gname]) for gname, _ in LAYER_GROUPS}
+        del host_groups
         self.copies = [base] + [{k: tuple(t.clone() for t in v) for k, v in base.items()}
                                 for _ in range(1, n_copies)]
         # per layer group and pass: activations and outputs, each a view of one
@@ -231,8 +252,7 @@ class DecodeWorkload:
         ox = oy = 0
         for gi, gname, mode, M, N, K, g in shapes:
             xh = self.x_flat_host[ox:ox + M * K].view(M, K)
-            xh.copy_(torch.from_numpy(synth.activations(synth.SEED_ACTS + 10 * gi + 100 * mode,
-                                                        M, K)))
+            xh.copy_(torch.from_numpy(host_acts[gname, mode]))
             self.x_host[gname, mode] = xh
             self.x[gname, mode] = self.x_flat[ox:ox + M * K].view(M, K)
             b = self._bufs(M, N, K, g)
@@ -301,6 +321,15 @@ class DecodeWorkload:
                     events[gname, mode][1].record()
         if e2e:  # and every output back in one download
             self.y_flat_host.copy_(self.y_flat, non_blocking=True)
+
+    def step_results(self):
+        """Host copies of the step's results, per (group, pass): output y,
+        int8 activation codes and their fp32 scales."""
+        import torch
+
+        torch.cuda.synchronize()
+        return {k: (b["y"].cpu().numpy(), b["xq"].cpu().numpy(), b["xs"].cpu().numpy())
+                for k, b in self.bufs.items()}
 
     def run_projection(self, name, mode):
         """One unfused projection: quantise its own input and apply the layer."""
@@ -406,30 +435,73 @@ def measure_prefill(wl, reps=10):
 
 
 # -------------------------------------------------------------- CPU oracle
-def cpu_baseline(rows_per_proj=256, budget_s=20.0):
-    """The oracle, as it stands, on the host cores: every projection and both
-    passes of the step on a sample of output rows, scaled to the whole step."""
+def oracle_step_inputs():
+    """The step's inputs as the oracle takes them: packed planes per group."""
+    import oracle
+
+    groups, acts = step_host_inputs()
+    packed = {g: (oracle.pack_plane(uh), oracle.pack_plane(ul), s)
+              for g, (uh, ul, s) in groups.items()}
+    return packed, acts
+
+
+def oracle_step(packed, acts):
+    """One decode step by the oracle: per (group, pass) (y, codes, scales)."""
+    import oracle
+
+    outs = {}
+    for gname, members in LAYER_GROUPS:
+        N, K, g = group_shape(members)
+        hi, lo, s = packed[gname]
+        for mode in DECODE_M:
+            q, xs = oracle.quantize(acts[gname, mode], g)
+            outs[gname, mode] = (oracle.linear(mode, hi, lo if mode else None, s, q, xs, K, g),
+                                 q, xs)
+    return outs
+
+
+def compare_step(outs, results, tol=1e-3):
+    """The GPU step's results against the oracle's: activation codes and
+    scales bit-exact, every output element within `tol` in the normalised
+    error max |y - y_ref| / (|y_ref| + 1e-3 rms(y_ref)).  "ok" or the list
+    of failures."""
+    import oracle
+
+    bad = []
+    for key, (y_ref, q, xs) in outs.items():
+        y, xq_gpu, xs_gpu = results[key]
+        tag = f"{key[0]}/{'draft' if key[1] == 0 else 'target'}"
+        if not (np.array_equal(xq_gpu, q) and np.array_equal(xs_gpu, xs)):
+            bad.append(f"{tag}: activation codes differ")
+        err = oracle.max_normalised_error(y, y_ref) if y.shape == y_ref.shape else float("inf")
+        if not err <= tol:
+            bad.append(f"{tag}: output error {err:.3g}")
+    return "ok" if not bad else "FAILED: " + "; ".join(bad)
+
+
+def cpu_baseline(results=None, budget_s=12.0, max_steps=None):
+    """The oracle, as it stands, on the host cores: whole decode steps (every
+    layer group, both passes, every output row) on the step's own seeded
+    inputs, repeated until `budget_s` of CPU work (at least one step, at most
+    `max_steps`).  Returns (seconds per step, threads, steps, self_check).
+
+    With `results` (the GPU step's outputs, from DecodeWorkload.step_results)
+    the first oracle step also checks them (compare_step)."""
     import oracle
 
     oracle.build()
-    t_total = 0.0
-    sampled = 0
-    for name, (N, K, g) in synth.LLAMA3_8B_PROJECTIONS.items():
-        pid = synth.PROJ_IDS[name]
-        rows = min(rows_per_proj, N)
-        uh = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_HI, N, K, 0, rows)
-        ul = synth.nibbles(synth.SEED_WEIGHTS + pid, synth.STREAM_LO, N, K, 0, rows)
-        s = synth.group_scales(synth.SEED_SCALES + pid, N, K, 0, rows)
-        hi, lo = oracle.pack_plane(uh), oracle.pack_plane(ul)
-        for mode, M in DECODE_M.items():
-            x = synth.activations(synth.SEED_ACTS + pid + 100 * mode, M, K)
-            t0 = time.perf_counter()
-            q, xs = oracle.quantize(x, g)
-            oracle.linear(mode, hi, lo if mode else None, s, q, xs, K, g)
-            dt = time.perf_counter() - t0
-            t_total += dt * (N / rows)  # scale the row sample to the full projection
-            sampled += rows
-    return t_total, oracle.num_threads(), sampled
+    packed, acts = oracle_step_inputs()
+    check = None
+    times = []
+    while True:
+        t0 = time.perf_counter()
+        outs = oracle_step(packed, acts)
+        times.append(time.perf_counter() - t0)
+        if results is not None and len(times) == 1:
+            check = compare_step(outs, results)
+        if sum(times) >= budget_s or (max_steps is not None and len(times) >= max_steps):
+            break
+    return statistics.median(times), oracle.num_threads(), len(times), check
 
 
 def measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind):
@@ -901,6 +973,7 @@ def main():
     dec = None
     if args.workload in ("all", "decode"):
         dec = measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind)
+        step_results = wl.step_results()
     sweep = rnd = None
     if args.workload in ("all", "sweep"):
         sweep = measure_sweep(wl, hbm_peak, reps=5 if args.workload == "all" else 2)
@@ -993,13 +1066,16 @@ def main():
     if spec_res is not None:
         out["speculative_rounds"] = spec_res
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_cpu, cores, rows = cpu_baseline()
+        t_cpu, cores, n_steps, check = cpu_baseline(results=step_results)
         out["cpu_baseline"] = {
             "value": round(step_bytes / t_cpu / 1e9, 4), "unit": UNIT, "cores": cores,
             "kind": "oracle",
-            "sample": f"every projection, both passes, first {rows // 14} output rows each "
-                      f"({rows} row-passes), time scaled by N/rows to one full step",
+            "sample": f"{n_steps} whole decode steps on the step's own inputs (every layer "
+                      "group, both passes, every output row), median step time",
         }
+        out["self_check"] = check
+    else:
+        out["self_check"] = "not run (no oracle leg on this rank or run)"
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -1048,14 +1124,10 @@ def run_reference(args, rank, world, wl_name):
     if rank != 0:
         return
     step_bytes = decode_step_bytes()
-    rows = 64
-    for _ in range(min(args.warmup, 1)):
-        cpu_baseline(rows_per_proj=rows)
-    times = []
-    for _ in range(args.steps if args.steps <= 5 else 5):
-        t, cores, sampled = cpu_baseline(rows_per_proj=rows)
-        times.append(t)
-    t = statistics.median(times)
+    steps = min(args.steps, 60)  # whole oracle steps: about 0.7 s each on 16 threads
+    cpu_baseline(budget_s=0.0, max_steps=1)  # warm-up (first-touch of the inputs)
+    t, cores, n, _ = cpu_baseline(budget_s=float("inf"), max_steps=steps)
+    times = [t] * n
     value = step_bytes / t / 1e9
     out = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
@@ -1066,8 +1138,8 @@ def run_reference(args, rank, world, wl_name):
         "timing": "host wall clock of the oracle, median over the steps",
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"first {rows} output rows of every projection and pass, "
-                                   "scaled by N/rows to one full step"},
+                         "sample": f"{n} whole decode steps (every layer group, both passes, "
+                                   "every output row), median step time"},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
