@@ -43,9 +43,10 @@
 //          group (from the landed activation tile)
 //   4      TMA producer: activation tile (128-byte swizzle) and the hi / lo
 //          plane tiles of the group, one mbarrier per stage (this CTA only)
-//   5      TMEM owner and MMA issuer (one thread)
-//   6, 7   per-group constants, batches in turn: row scales, per-token
-//          constants c (and the per-group activation scales for o_proj)
+//   5, 6   MMA issuers (one thread each), even and odd groups; warp 5 owns
+//          the tensor memory
+//   7      per-group constants: row scales, per-token constants c (and the
+//          per-group activation scales for o_proj)
 //   8..15  epilogue: TMEM -> registers -> fp32 running sums (two warps per
 //          TMEM lane quarter, half of the tokens each)
 // The other warpgroups hand registers to the epilogue (setmaxnreg), which
@@ -67,7 +68,14 @@ constexpr int BW = 128;  // weight rows per tile
 constexpr int kMaxStages = 8;
 constexpr int kWarpXf0 = 0, kNumXf = 4;  // one warpgroup
 constexpr int kXfThreads = 32 * kNumXf;
-constexpr int kWarpTma = kNumXf, kWarpMma = kNumXf + 1, kWarpPrep0 = kNumXf + 2, kNumPrep = 2;
+// two MMA issuers on alternate groups: one thread issues an MMA only every
+// ~50 cycles, about as long as the tensor core takes to run one of 128 x 128
+// x 32, so a single issuer with its waits between groups cannot keep it busy
+constexpr int kWarpTma = kNumXf, kWarpMma0 = kNumXf + 1, kNumMma = 2;
+constexpr int kWarpPrep = kNumXf + 3;
+// groups' MMA completion: one barrier per group in a ring whose length is a
+// multiple of the stage count (2, 3 or 4) and of the accumulator count (3)
+constexpr int kDone = 12;
 constexpr int kWarpEpi0 = kNumXf + 4, kNumEpi = 8;  // two epilogue warps per TMEM lane quarter
 constexpr int kWarps = kWarpEpi0 + kNumEpi;
 constexpr int kThreads = kWarps * 32;
@@ -151,9 +159,13 @@ __host__ __device__ constexpr int cslot_bytes(int bt) { return BW * 4 + 2 * bt *
 
 __host__ __device__ constexpr int cslots(int) { return 16; }
 
+// mbarriers: fullB, fullA [kMaxStages each], done [kDone], fullC, emptyC
+// [16 each], accEmpty [4]
+constexpr int kBarriers = 2 * kMaxStages + kDone + 2 * 16 + 4;
+
 __host__ __device__ constexpr int smem_total(int mode, int bt, int stages) {
-  return 1024 + stages * stage_bytes(mode, bt) + cslots(bt) * cslot_bytes(bt) +
-         (3 * kMaxStages + 2 * 16 + 2 * 4) * 8 + 16;
+  return 1024 + stages * stage_bytes(mode, bt) + cslots(bt) * cslot_bytes(bt) + kBarriers * 8 +
+         16;
 }
 
 // d = a * b + c on float pairs (one packed f32x2 instruction).
@@ -196,12 +208,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sXv = [&](int c) { return reinterpret_cast<float *>(sCv(c) + BT); };
   uint64_t *bars = reinterpret_cast<uint64_t *>(cbase + CS * CSLOT);
   uint64_t *fullB = bars;                      // activation and plane tiles landed
-  uint64_t *fullA = bars + kMaxStages;         // byte operand written
-  uint64_t *stageFree = bars + 2 * kMaxStages; // MMAs done with the stage
-  uint64_t *fullC = bars + 3 * kMaxStages;     // [CS] per-group constants written
+  uint64_t *fullA = bars + kMaxStages;         // byte operand written (the tiles landed)
+  uint64_t *done = bars + 2 * kMaxStages;      // [kDone] the group's MMAs complete:
+                                               // stage and accumulator readable / free
+  uint64_t *fullC = done + kDone;              // [CS] per-group constants written
   uint64_t *emptyC = fullC + CS;               // [CS] epilogue done with them
-  uint64_t *accFull = emptyC + CS;             // [NACC] accumulator ready
-  uint64_t *accEmpty = accFull + NACC;         // [NACC] accumulator drained and re-seeded
+  uint64_t *accEmpty = emptyC + CS;            // [NACC] accumulator read out
   uint32_t *tslot = reinterpret_cast<uint32_t *>(accEmpty + NACC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -210,19 +222,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&fullB[s], 1);
       mbar_init(&fullA[s], kNumXf);
-      mbar_init(&stageFree[s], 1);
     }
     for (int c = 0; c < CS; ++c) {
       mbar_init(&fullC[c], XS ? 1 + kNumXf : 1);  // one prep warp per slot
       mbar_init(&emptyC[c], kNumEpi);
     }
-    for (int b = 0; b < NACC; ++b) {
-      mbar_init(&accFull[b], 1);
-      mbar_init(&accEmpty[b], kNumEpi);
-    }
+    for (int d = 0; d < kDone; ++d) mbar_init(&done[d], 1);
+    for (int b = 0; b < NACC; ++b) mbar_init(&accEmpty[b], kNumEpi);
     fence_barrier_init();
   }
-  if (warp == kWarpMma) {
+  if (warp == kWarpMma0) {
     tmem_alloc(tslot, TCOLS);
     tmem_relinquish();
   }
@@ -332,40 +341,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_hi);
       if (MODE) prefetch_tmap(&tm_lo);
       griddep_wait();
-      int it = 0, s = 0;
-      uint32_t ph = 0;
+      int it = 0, s = 0, fd = 0;  // fd: done slot of group it - S
+      uint32_t fdph = 0;
       bool ok = true;
       constexpr uint32_t bytes = BT * 128 + BW * 64 * (MODE ? 2 : 1);
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
         const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
         const int n0 = tc.n0, m0 = tc.m0;
         for (int g = tc.g0; g < tc.g1; ++g, ++it) {
-          if (!mbar_wait(&stageFree[s], ph ^ 1u)) {
-            ok = false;
-            break;
+          if (it >= S) {  // the stage's previous group: its MMAs are complete
+            if (!mbar_wait(&done[fd], fdph)) {
+              ok = false;
+              break;
+            }
+            if (++fd == kDone) {
+              fd = 0;
+              fdph ^= 1u;
+            }
           }
           mbar_arrive_expect_tx(&fullB[s], bytes);
           tma_load_2d(sB(s), &tm_q, &fullB[s], g * 128, m0);
           tma_load_2d(sH(s), &tm_hi, &fullB[s], g * 64, n0);
           if (MODE) tma_load_2d(sL(s), &tm_lo, &fullB[s], g * 64, n0);
-          if (++s == S) {
-            s = 0;
-            ph ^= 1u;
-          }
+          if (++s == S) s = 0;
         }
       }
       if (!ok)  // gave up: let the copies already issued land
         for (int i = (it > S ? it - S : 0); i < it; ++i)
           mbar_wait_final(&fullB[i % S], (i / S) & 1);
     }
-    } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
+    } else if (warp < kWarpMma0 + kNumMma) {
+    // ----------------------------------------------------------- MMA issuers
+    // issuer i takes the groups it = i, i + 2, ...: it waits for the group's
+    // operand (written after the tiles landed, so it implies them) and its
+    // accumulator, issues the four MMAs and one commit that tells the TMA
+    // producer (stage free) and the epilogue (accumulator full).  Counts,
+    // slots and phases are kept incrementally for every group.
     if (lane == 0) {
-      // every count, slot and descriptor is kept incrementally: this one
-      // thread shares its scheduler with busy warps, so each instruction it
-      // saves shortens the gap between two groups' MMAs
-      int s = 0, b = 0, lb = 0;
-      uint32_t ph = 0, bph = 0, lbph = 0;
+      const int mine = warp - kWarpMma0;
+      int it = 0, s = 0, b = 0, d = 0, ld = 0;
+      uint32_t ph = 0, bph = 0, dph = 0, ldph = 0;
       bool issued = false;
       const uint64_t bd0 = umma_desc_sw128(sB(0));
       const uint32_t at0 = tmem + (uint32_t)tmem_abase(BT);  // the weight operand slots
@@ -373,22 +388,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
         const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
-        for (int g = tc.g0; g < tc.g1; ++g) {
-          ok = mbar_wait(&fullB[s], ph) && mbar_wait(&fullA[s], ph) &&
-               mbar_wait(&accEmpty[b], bph ^ 1u);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t bd = bd0 + (uint64_t)s * kStageDesc;
-          const uint32_t at = at0 + (uint32_t)(32 * s);
-          const uint32_t dt = tmem + (uint32_t)(b * BT);
+        for (int g = tc.g0; g < tc.g1; ++g, ++it) {
+          if ((it & 1) == mine) {
+            ok = mbar_wait(&fullA[s], ph) && mbar_wait(&accEmpty[b], bph ^ 1u);
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t bd = bd0 + (uint64_t)s * kStageDesc;
+            const uint32_t at = at0 + (uint32_t)(32 * s);
+            const uint32_t dt = tmem + (uint32_t)(b * BT);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // 4 x K=32: 8 TMEM columns of A, 32 bytes of B
-            umma_i8_ta(dt, at + 8 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
-          umma_commit(&stageFree[s]);
-          umma_commit(&accFull[b]);
-          issued = true;
-          lb = b;
-          lbph = bph;
+            for (int kk = 0; kk < 4; ++kk)  // 4 x K=32: 8 TMEM columns of A, 32 bytes of B
+              umma_i8_ta(dt, at + 8 * kk, bd + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
+            umma_commit(&done[d]);
+            issued = true;
+            ld = d;
+            ldph = dph;
+          }
           if (++s == S) {
             s = 0;
             ph ^= 1u;
@@ -397,32 +412,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             b = 0;
             bph ^= 1u;
           }
+          if (++d == kDone) {
+            d = 0;
+            dph ^= 1u;
+          }
         }
       }
-      // every MMA issued must be complete before TMEM is released (also
-      // after a wait gave up): commits complete in order
-      if (issued) mbar_wait_final(&accFull[lb], lbph);
+      // every MMA this thread issued must be complete before TMEM is released
+      // (also after a wait gave up): its commits complete in order
+      if (issued) mbar_wait_final(&done[ld], ldph);
     }
-    } else if (warp >= kWarpPrep0) {
+    } else if (warp == kWarpPrep) {
     // ----------------------------------------------- per-group constants
     // CBATCH groups per round trip: lane i holds rows i + 32 r (r < 4) and
     // tokens i + 32 u (u < BT / 32, at least one), all loads of a batch
-    // issued before the first use.  Two warps take turns batch by batch, so
-    // two round trips are in flight.
+    // issued before the first use.
     constexpr int TU = BT < 32 ? 1 : BT / 32;
     constexpr int CB = C::CBATCH;
-    const int pw = warp - kWarpPrep0;
     griddep_wait();
-    int it = 0, batch = 0;
+    int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
       const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
       const int n0 = tc.n0, m0 = tc.m0, G1 = tc.g1, G = p.G;
-      for (int gb = tc.g0; gb < G1 && ok; gb += CB, ++batch) {
-        if (batch % kNumPrep != pw) {  // the other warp's batch
-          it += min(CB, G1 - gb);
-          continue;
-        }
+      for (int gb = tc.g0; gb < G1 && ok; gb += CB) {
         uint16_t sv[4][CB];
         int rv[TU][CB];
         float xv[TU][CB];
@@ -493,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) continue;  // after a give-up: no more waits, but every tile still arrives below
         const int cs = it % CS, b = it % NACC;
         ok = mbar_wait_warp(&fullC[cs], (it / CS) & 1) &&
-             mbar_wait_warp(&accFull[b], (it / NACC) & 1);
+             mbar_wait_warp(&done[it % kDone], (it / kDone) & 1);
         if (!ok) continue;
         tc_fence_after();
         const float sg = sSg(cs)[row];
@@ -597,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == kWarpMma0) {
     tc_fence_after();
     tmem_dealloc(tmem, TCOLS);
   }
