@@ -337,3 +337,23 @@ def test_quantize_linear_without_group_sums(M, N, K, mode):
         assert np.array_equal(host(xq), p.q) and np.array_equal(host(xs), p.xs)
         assert oracle.max_normalised_error(host(y), p.y_ref(mode)) <= TOL
     assert bn.device_wait_timeout(reset=True) == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (4, 28672, 4096), (4, 4096, 14336),
+                                   (8, 300, 1024), (2, 1024, 2048)])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("act_group", [0, 128])
+def test_one_launch_quantise_and_apply_equals_two_steps(M, N, K, mode, act_group):
+    """On the decode GEMV (with programmatic dependent launch) the one-call
+    entry gives, bit for bit, the codes, scales, sums and output of the
+    quantiser followed by the layer."""
+    p = Problem(M, N, K, seed=11 * M + K, act_group=act_group)
+    y1, (q1, s1, u1) = bn.quantize_linear(mode, p.d_hi, p.d_lo, p.d_s, p.d_x, act_group,
+                                          path=bn.PATH_GEMV | bn.PATH_OVERLAP)
+    q2, s2, u2 = bn.quantize_act(p.d_x, act_group)
+    y2 = bn.linear(mode, p.d_hi, p.d_lo, p.d_s, q2, s2, u2, act_group, path=bn.PATH_GEMV)
+    torch.cuda.synchronize()
+    assert torch.equal(q1, q2) and torch.equal(s1, s2) and torch.equal(u1, u2)
+    assert torch.equal(y1, y2)
+    assert np.array_equal(host(q1), p.q)
+    assert bn.device_wait_timeout(reset=True) == 0
