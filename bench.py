@@ -702,11 +702,13 @@ def attention_bytes(mode, H, Hkv, T, D=128):
     return planes + 2 * 2 * rows + 2 * H * D + 4 * H * D
 
 
-def measure_attention(wl, hbm_peak, reps=20):
+def measure_attention(wl, hbm_peak, reps=10, chain=20):
     """bitnest_nested_attention for one Llama-3-8B decode token (32 query
     heads, 8 KV heads, head_dim 128) over caches of 2048 and 8192 tokens
     (seeded synthetic K / V packed with bitnest_pack_weights), draft (KV4) and
-    target (KV8); one launch after a spin, CUDA events."""
+    target (KV8).  Device time per launch: a CUDA graph of `chain` launches
+    back to back, CUDA events around its replay (so the per-launch time
+    includes the gap between two launches, not the events' own cost)."""
     import torch
 
     bn = wl.bn
@@ -722,16 +724,19 @@ def measure_attention(wl, hbm_peak, reps=20):
         q = torch.randn((H, D), generator=gen, device=wl.dev).half()
         out = torch.empty((H, D), dtype=torch.float32, device=wl.dev)
         for mode in (0, 1):
-            bn.nested_attention(mode, q, kp, vp, Hkv, out=out)
-            t = 0.0
+            g = capture(lambda: [bn.nested_attention(mode, q, kp, vp, Hkv, out=out)
+                                 for _ in range(chain)])
+            g.replay()
+            torch.cuda.synchronize()
+            ts = []
             for _ in range(reps):
-                torch.cuda._sleep(200_000)
                 a.record()
-                bn.nested_attention(mode, q, kp, vp, Hkv, out=out)
+                g.replay()
                 b.record()
                 torch.cuda.synchronize()
-                t += a.elapsed_time(b) / 1e3
-            t /= reps
+                ts.append(a.elapsed_time(b) / 1e3 / chain)
+            g.reset()
+            t = statistics.median(ts)
             nb = attention_bytes(mode, H, Hkv, T, D)
             res[f"{'draft' if mode == 0 else 'target'}/T={T}"] = {
                 "us": round(t * 1e6, 2), "GB/s": round(nb / t / 1e9, 1),
@@ -739,6 +744,7 @@ def measure_attention(wl, hbm_peak, reps=20):
         del kv, kp, vp
     return {"workload": "decode attention of one token over a nested KV cache (H=32, Hkv=8, "
                         "D=128), draft reads KV4 (hi planes), target KV8 (hi + lo)",
+            "timing": f"CUDA graph of {chain} launches, median of {reps} replays, per launch",
             "per_case": res}
 
 
