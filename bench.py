@@ -607,24 +607,61 @@ SWEEP_M = (1, 2, 4, 8, 16, 32, 64, 128)
 SWEEP_SHAPES = ("gate_proj", "down_proj")  # 14336 x 4096 and 4096 x 14336
 
 
+def weight_copies(wl, N, K, nbytes, min_copies=3, max_copies=64):
+    """Rotating copies of seeded [N, K] planes and scales, enough that between
+    two reads of one copy the others push it out of the 126 MB L2."""
+    import torch
+
+    bn = wl.bn
+    count = max(min_copies, min(max_copies, -(-160_000_000 // max(nbytes, 1)) + 1))
+    uh = torch.from_numpy(synth.nibbles(synth.SEED_WEIGHTS + 50 + N, synth.STREAM_HI, N, K)).to(wl.dev)
+    ul = torch.from_numpy(synth.nibbles(synth.SEED_WEIGHTS + 50 + N, synth.STREAM_LO, N, K)).to(wl.dev)
+    sc = torch.from_numpy(synth.group_scales(synth.SEED_SCALES + 50 + N, N, K)).to(wl.dev)
+    hi, lo = bn.pack_planes(uh, ul)
+    del uh, ul
+    return [(hi, lo, sc)] + [(hi.clone(), lo.clone(), sc.clone()) for _ in range(count - 1)]
+
+
+def chained(fn_of_copy, copies, reps=8, per_copy=2):
+    """Device time per launch of `fn_of_copy(c)`: a CUDA graph of
+    len(copies) * per_copy launches cycling over the copies, CUDA events
+    around each replay, median over `reps` replays."""
+    import torch
+
+    n = len(copies) * per_copy
+    g = capture(lambda: [fn_of_copy(i % len(copies)) for i in range(n)])
+    g.replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(reps):
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / 1e3 / n)
+    g.reset()
+    return statistics.median(ts)
+
+
 def measure_sweep(wl, hbm_peak, reps=5):
     """Every M of the batch / verify sweep on the two MLP shapes, both modes:
-    the path the library picks, device time per launch (CUDA events around the
-    launch, after a 256 MB L2 flush), HBM throughput and int8 TOPS."""
+    the path the library picks, device time per launch from a CUDA graph of
+    back-to-back launches over rotating weight copies (each launch reads its
+    weights from HBM; the time includes the gap between two launches but not
+    the events' own cost), HBM throughput and int8 TOPS."""
     import torch
 
     bn = wl.bn
     dev = wl.dev
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
     res = {}
     torch.cuda._sleep(200_000_000)  # about 0.1 s of spinning: clocks up before the first case
     torch.cuda.synchronize()
     for name in SWEEP_SHAPES:
         N, K, g = synth.LLAMA3_8B_PROJECTIONS[name]
-        hi, lo, sc = wl.single[name]
         pid = synth.PROJ_IDS[name]
+        copies = weight_copies(wl, N, K, N * K // 2, min_copies=6)
         for M in SWEEP_M:
             x = torch.from_numpy(synth.activations(synth.SEED_ACTS + pid + 1000 * M, M, K)).to(dev)
             xq, xs, xsum = bn.quantize_act(x, g)
@@ -634,16 +671,8 @@ def measure_sweep(wl, hbm_peak, reps=5):
                 # scratch for the tensor-core path's split K (few tiles, long K)
                 nws = bn.linear_ws_bytes(mode, M, N, K)
                 ws = bn.workspace(nws, dev) if nws else None
-                bn.linear_ws(mode, hi, lo, sc, xq, xs, xsum, ws, g, out=y)  # warm
-                t = 0.0
-                for _ in range(reps):
-                    flush.fill_(1)
-                    a.record()
-                    bn.linear_ws(mode, hi, lo, sc, xq, xs, xsum, ws, g, out=y)
-                    b.record()
-                    torch.cuda.synchronize()
-                    t += a.elapsed_time(b) / 1e3
-                t /= reps
+                t = chained(lambda c: bn.linear_ws(mode, *copies[c], xq, xs, xsum, ws, g, out=y),
+                            copies, reps=reps)
                 nb = linear_bytes(mode, M, N, K)
                 label = "tcgen05 split-K" if nws else (
                     "gemv" if path == bn.PATH_GEMV else "tcgen05")
@@ -653,8 +682,55 @@ def measure_sweep(wl, hbm_peak, reps=5):
                     "frac_hbm": round(nb / t / 1e9 / hbm_peak, 3),
                     "TOPS": round(2.0 * M * N * K / t / 1e12, 2)}
             del x, xq, xs, xsum, y
-    del flush
+        del copies
     return res
+
+
+def measure_call_cost(wl, hbm_peak, reps=5):
+    """Fixed cost per decode call: t = a + bytes / BW fitted (least squares)
+    over K = 4096 layers of N = 1024, 4096, 14336 and 28672 rows, draft
+    (M = 1) and target (M = 4), for the layer alone (`bitnest_linear` on
+    quantised activations) and for the one-call quantise + layer entry
+    (`bitnest_quantize_linear`, the decode step's call).  Device time per
+    launch from CUDA graphs over rotating weight copies (`chained`)."""
+    import torch
+
+    bn = wl.bn
+    dev = wl.dev
+    K, g = 4096, 0
+    P = bn.PATH_AUTO | bn.PATH_OVERLAP
+    pts = {}
+    for N in (1024, 4096, 14336, 28672):
+        copies = weight_copies(wl, N, K, N * K // 2)
+        for mode, M in DECODE_M.items():
+            x = torch.from_numpy(synth.activations(synth.SEED_ACTS + 900 + M, M, K)).to(dev)
+            xq, xs, _ = bn.quantize_act(x, g)
+            ao = (torch.empty_like(xq), torch.empty_like(xs), None)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            t_lin = chained(lambda c: bn.linear(mode, *copies[c], xq, xs, None, g, out=y, path=P),
+                            copies, reps=reps)
+            t_ql = chained(lambda c: bn.quantize_linear(mode, *copies[c], x, g, out=y, act_out=ao,
+                                                        path=P), copies, reps=reps)
+            tag = "draft" if mode == 0 else "target"
+            pts.setdefault(("layer", tag), []).append((linear_bytes(mode, M, N, K), t_lin, N))
+            pts.setdefault(("quantise+layer", tag), []).append(
+                (fused_bytes(mode, M, N, K, g), t_ql, N))
+        del copies
+    res = {}
+    for (kind, tag), v in pts.items():
+        xb = np.array([b for b, _, _ in v], np.float64)
+        yt = np.array([t for _, t, _ in v], np.float64)
+        slope, icpt = np.polyfit(xb, yt, 1)
+        res[f"{kind}/{tag}"] = {
+            "a_us": round(icpt * 1e6, 2), "BW_GB/s": round(1.0 / slope / 1e9, 1),
+            "BW_frac_hbm": round(1.0 / slope / 1e9 / hbm_peak, 3),
+            "points": {f"N={n}": {"MB": round(b / 1e6, 2), "us": round(t * 1e6, 2),
+                                  "frac_hbm": round(b / t / 1e9 / hbm_peak, 3)}
+                       for b, t, n in v}}
+    return {"workload": "decode calls on K = 4096 layers (N = 1024 .. 28672), draft M = 1, "
+                        "target M = 4; fit t = a + bytes / BW",
+            "timing": "CUDA graph of back-to-back calls over rotating weight copies, per call",
+            "per_kind": res}
 
 
 # ------------------------------------------- down_proj input: R4 rotation
@@ -942,8 +1018,8 @@ def main():
                     help="launch the step's kernels directly instead of replaying a CUDA graph "
                          "(for profilers that cannot replay the captured kernel nodes)")
     ap.add_argument("--workload", default="all",
-                    choices=["all", "decode", "prefill", "sweep", "round", "pack", "hadamard",
-                             "attention", "spec"],
+                    choices=["all", "decode", "prefill", "sweep", "cost", "round", "pack",
+                             "hadamard", "attention", "spec"],
                     help="all: the decode step line with the prefill, M-sweep and "
                          "decode-round objects; otherwise only that part (profiling runs)")
     args = ap.parse_args()
@@ -980,9 +1056,11 @@ def main():
     if args.workload in ("all", "decode"):
         dec = measure_decode(args, wl, barrier, max_over_ranks, world, hbm_peak, peak_kind)
         step_results = wl.step_results()
-    sweep = rnd = None
+    sweep = rnd = cost = None
     if args.workload in ("all", "sweep"):
         sweep = measure_sweep(wl, hbm_peak, reps=5 if args.workload == "all" else 2)
+    if args.workload in ("all", "cost"):
+        cost = measure_call_cost(wl, hbm_peak, reps=5 if args.workload == "all" else 3)
     if args.workload in ("all", "round"):
         rnd = measure_round(wl, hbm_peak, reps=10 if args.workload == "all" else 3)
     pack = None
@@ -1024,7 +1102,8 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         if rank == 0:
-            part = {"prefill": prefill, "m_sweep": sweep, "decode_round": rnd,
+            part = {"prefill": prefill, "m_sweep": sweep, "decode_call_cost": cost,
+                    "decode_round": rnd,
                     "pack_from_weights": pack, "down_proj_input_rotation": had,
                     "nested_kv_attention": att, "speculative_rounds": spec_res}
             print(json.dumps({"metric": METRIC, "workload": f"{args.workload} only",
@@ -1059,8 +1138,12 @@ def main():
         out["prefill"] = prefill
     if sweep is not None:
         out["m_sweep"] = {"workload": "M in {1..128} x gate_proj 14336x4096 / down_proj "
-                                      "4096x14336 x draft / target, one launch after an L2 flush",
+                                      "4096x14336 x draft / target",
+                          "timing": "CUDA graph of back-to-back launches over six rotating "
+                                    "weight copies (weights read from HBM), per launch",
                           "per_case": sweep}
+    if cost is not None:
+        out["decode_call_cost"] = cost
     if rnd is not None:
         out["decode_round"] = rnd
     if pack is not None:

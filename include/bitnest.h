@@ -159,8 +159,14 @@ int bitnest_hadamard_quantize_act(const uint16_t *x, int64_t M, int64_t K, int8_
  *   out                 : fp32 [H, D];  head h attends with KV head
  *                         h / (H / Hkv):  softmax(q K^T / sqrt(D)) V.
  * D must be 128, H / Hkv one of 1, 2, 4, 8, T >= 1 (else
- * BITNEST_ERR_UNSUPPORTED_SHAPE).  fp32 arithmetic: agrees with an exact
- * evaluation to fp32 rounding.
+ * BITNEST_ERR_UNSUPPORTED_SHAPE).  Both products run on the tensor cores with
+ * fp16 operands that are exact (the queries as given, the integer codes) and
+ * fp32 accumulation; the scales and the softmax are fp32, and p * v_scale
+ * enters as two fp16 terms (22 bits): within 1e-3 of an exact evaluation in
+ * the normalised error max |out - ref| / (|ref| + 1e-3 rms(ref)).  One launch:
+ * the tokens of each KV head are split over a thread-block cluster of up to
+ * 16 CTAs (8 where the device cannot place 16), merged in the cluster's
+ * shared memory; nothing is allocated, no scratch is needed.
  */
 int bitnest_nested_attention(int mode, const uint16_t *q, int64_t H, int64_t Hkv, int64_t D,
                              int64_t T, const uint8_t *k_hi, const uint8_t *k_lo,
