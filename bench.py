@@ -734,10 +734,12 @@ def measure_call_cost(wl, hbm_peak, reps=5):
 
 
 # ------------------------------------------- down_proj input: R4 rotation
-def measure_hadamard(wl, hbm_peak, reps=20):
+def measure_hadamard(wl, hbm_peak, reps=10, chain=20):
     """bitnest_hadamard_quantize_act (x H / sqrt(K) + per-token int8) on the
     down_proj input (K = 14336) next to the plain quantiser, at the decode
-    batches and the prefill batch; one launch after a spin, CUDA events."""
+    batches and the prefill batch.  Device time per launch: a CUDA graph of
+    `chain` launches back to back (the decode-size rows stay in L2, as they
+    would coming from the preceding kernel), CUDA events around each replay."""
     import torch
 
     bn = wl.bn
@@ -747,28 +749,34 @@ def measure_hadamard(wl, hbm_peak, reps=20):
     res = {}
     for M in (1, 4, PREFILL_M):
         x = torch.from_numpy(synth.activations(synth.SEED_ACTS + 500 + M, M, K)).to(wl.dev)
+        out = (torch.empty((M, K), dtype=torch.int8, device=wl.dev),
+               torch.empty((M,), dtype=torch.float32, device=wl.dev),
+               torch.empty((M, K // 128), dtype=torch.int32, device=wl.dev))
         nbytes = 2 * M * K + M * K + 4 * M + 4 * M * (K // 128)
-        for name, fn in (("rotate+quantise", lambda: bn.hadamard_quantize_act(x)),
-                         ("quantise", lambda: bn.quantize_act(x, 0))):
-            fn()
-            t = 0.0
+        n = chain if M < PREFILL_M else 4
+        for name, fn in (("rotate+quantise", lambda: bn.hadamard_quantize_act(x, out=out)),
+                         ("quantise", lambda: bn.quantize_act(x, 0, out=out))):
+            g = capture(lambda: [fn() for _ in range(n)])
+            g.replay()
+            torch.cuda.synchronize()
+            ts = []
             for _ in range(reps):
-                torch.cuda._sleep(200_000)
                 a.record()
-                fn()
+                g.replay()
                 b.record()
                 torch.cuda.synchronize()
-                t += a.elapsed_time(b) / 1e3
-            t /= reps
+                ts.append(a.elapsed_time(b) / 1e3 / n)
+            g.reset()
+            t = statistics.median(ts)
             res[f"{name}/M={M}"] = {"us": round(t * 1e6, 2), "GB/s": round(nbytes / t / 1e9, 1),
                                     "frac_hbm": round(nbytes / t / 1e9 / hbm_peak, 3)}
-        del x
+        del x, out
     return {"workload": "down_proj input (K = 14336 = 28 x 512): online Hadamard rotation "
                         "fused with per-token int8 quantisation, vs the quantiser alone",
+            "timing": f"CUDA graph of {chain} launches (4 at M = {PREFILL_M}), per launch",
             "per_case": res}
 
 
-# ------------------------------------------ nested KV cache: decode attention
 def attention_bytes(mode, H, Hkv, T, D=128):
     """Algorithmic bytes of one decode-attention launch: the K and V hi planes
     (and lo planes for the target) and their fp16 row scales, the fp16 query,

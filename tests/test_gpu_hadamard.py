@@ -66,3 +66,18 @@ def test_hadamard_quantize_then_down_proj_layer():
     y_ref = oracle.linear(1, oracle.pack_plane(uh), oracle.pack_plane(ul), s,
                           q_ref.astype(np.int8), xs_ref, K)
     assert oracle.max_normalised_error(host(y), y_ref) <= TOL
+
+
+def test_cluster_path_equals_one_cta_path():
+    """Decode sizes of K = 28 x 512 run on a 7-CTA cluster per token, larger
+    batches on one CTA per token; both take the same arithmetic in the same
+    order, so the codes, scales and sums of the same rows are identical."""
+    K = 14336
+    x = synth.activations(6200, 20, K)
+    x[3] = 0
+    small = [host(t) for t in bn.hadamard_quantize_act(dev(x[:5]))]  # cluster kernel
+    large = [host(t) for t in bn.hadamard_quantize_act(dev(x))]      # one CTA per token
+    torch.cuda.synchronize()
+    for a, b in zip(small, large):
+        assert np.array_equal(a, b[:5])
+    _check(x[:5])

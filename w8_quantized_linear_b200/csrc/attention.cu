@@ -98,6 +98,14 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+// distributed shared memory is used only once every CTA of the cluster has
+// started: each thread arrives at entry and waits before its first access
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
@@ -179,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 2) nested_attention_kernel(
   const int gid = lane >> 2, tig = lane & 3;
   const int c_begin = split * per_cta;
   const int c_end = min(T, c_begin + per_cta);
+  cluster_arrive();
   griddep_wait();  // q (and the cache) may come from the preceding kernel
   griddep_launch_dependents();
 
@@ -345,6 +354,7 @@ __global__ void __launch_bounds__(kThreads, 2) nested_attention_kernel(
     }
   }
   __syncthreads();
+  cluster_wait();  // every CTA of the cluster has started
   // this CTA's state, merged over its warps, into slot `split` of the first
   // CTA of the cluster
   const uint32_t rank = cluster_rank();

@@ -13,6 +13,14 @@
 // One CTA per token.  The row lives in shared memory in fp32 (K <= 32768);
 // the rotated row is quantised as the activation quantiser does (s =
 // max|x_rot| / 127, codes rne(x_rot / s)) with the group sums of the codes.
+//
+// Decode sizes of down_proj's K = 28 x 512 (a few tokens): one CTA per token
+// leaves the whole rotation to a single SM, so there a cluster of 7 CTAs
+// takes each token: CTA r transforms blocks 4 r .. 4 r + 3 and stores them
+// into every CTA of the cluster (distributed shared memory), mixes its own 4
+// output blocks from the full row, and the 7 partial maxima of |x_rot| meet
+// the same way before each CTA quantises its blocks.  The arithmetic is the
+// same, in the same order, as the one-CTA kernel's: the codes are identical.
 #include <math.h>
 
 #include "common.cuh"
@@ -201,6 +209,136 @@ __global__ void __launch_bounds__(kThreads) hadamard_quantize_kernel(
   }
 }
 
+// ----------------------------------------------- cluster kernel (K = 28 x 512)
+constexpr int kClusterCtas = 7;                 // CTAs per token
+constexpr int kBlocksPerCta = 28 / kClusterCtas;  // 4 blocks of 512
+constexpr int kCThreads = 256;
+constexpr int kClusterMaxM = 16;                // tokens up to which the cluster kernel is used
+
+__device__ __forceinline__ uint32_t cl_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// distributed shared memory is used only once every CTA of the cluster has
+// started: each thread arrives at entry and waits before its first access
+__device__ __forceinline__ void cl_arrive() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cl_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+// 16 bytes to the same shared-memory offset as `p` in CTA `rank` of the cluster
+__device__ __forceinline__ void st_cl4(float *p, uint32_t rank, float4 v) {
+  uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p)), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(ra), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_cl1(float *p, uint32_t rank, float v) {
+  uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p)), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+
+struct ClusterSmem {
+  float row[28 * 512];          // the transformed blocks of the whole row
+  float out[kBlocksPerCta * 512];  // this CTA's rotated output blocks
+  float amax[kClusterCtas];     // the CTAs' maxima of |x_rot|
+  float red[kCThreads / 32];
+};
+
+__global__ void __launch_bounds__(kCThreads) hadamard_quantize_cluster_kernel(
+    const uint16_t *__restrict__ x, float norm, int8_t *__restrict__ xq, float *__restrict__ xs,
+    int32_t *__restrict__ xsum) {
+  constexpr int K = 28 * 512, p = 512;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  ClusterSmem &sh = *reinterpret_cast<ClusterSmem *>(smem_raw);
+  const int64_t m = blockIdx.y;
+  const uint32_t rank = cl_rank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b0 = (int)rank * kBlocksPerCta;  // this CTA's blocks
+  cl_arrive();
+  griddep_wait();
+  griddep_launch_dependents();
+  // transform this CTA's blocks (one warp each) and store them into every CTA
+  if (warp < kBlocksPerCta)
+    fwht512_warp(x + m * K + (b0 + warp) * p, sh.out + warp * p, lane);  // staging
+  cl_wait();  // every CTA of the cluster has started
+  if (warp < kBlocksPerCta) {
+    const int blk = b0 + warp;
+    const float4 *v4 = reinterpret_cast<const float4 *>(sh.out + warp * p + 16 * lane);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = v4[q];
+      for (int r = 0; r < kClusterCtas; ++r)
+        st_cl4(sh.row + blk * p + 16 * lane + 4 * q, (uint32_t)r, v);
+    }
+  }
+  cl_sync();  // every CTA holds the whole transformed row
+  // mix: out[j][c] = sum_i H28[i][j] u[i][c] = total - 2 sum_{H28[i][j] < 0} u[i][c],
+  // for this CTA's output blocks j = b0 .. b0 + 3, then 1/sqrt(K)
+  constexpr H28Signs kSigns = h28_signs();
+  float amax = 0.0f;
+  for (int c = threadIdx.x; c < p; c += kCThreads) {
+    float u[28];
+    float total = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 28; ++i) {
+      u[i] = sh.row[i * p + c];
+      total += u[i];
+    }
+#pragma unroll
+    for (int jj = 0; jj < kBlocksPerCta; ++jj) {
+      const int j = b0 + jj;
+      float neg = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 28; ++i)
+        if ((kSigns.row[i] >> j) & 1u) neg += u[i];
+      const float o = (total - 2.0f * neg) * norm;
+      sh.out[jj * p + c] = o;
+      amax = fmaxf(amax, fabsf(o));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) sh.red[warp] = amax;
+  __syncthreads();
+  if (threadIdx.x < kClusterCtas) {  // this CTA's maximum into slot `rank` of every CTA
+    float a = sh.red[0];
+#pragma unroll
+    for (int w = 1; w < kCThreads / 32; ++w) a = fmaxf(a, sh.red[w]);
+    st_cl1(&sh.amax[rank], (uint32_t)threadIdx.x, a);
+  }
+  cl_sync();
+  amax = sh.amax[0];
+#pragma unroll
+  for (int r = 1; r < kClusterCtas; ++r) amax = fmaxf(amax, sh.amax[r]);
+  const float s = __fdiv_rn(amax, 127.0f);
+  const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
+  if (rank == 0 && threadIdx.x == 0) xs[m] = s;
+  // a warp per 128-column group of this CTA's blocks
+  constexpr int G = K / kGroup;
+  for (int gl = warp; gl < kBlocksPerCta * p / kGroup; gl += kCThreads / 32) {
+    const int g = b0 * (p / kGroup) + gl;
+    const float4 v = *reinterpret_cast<const float4 *>(sh.out + gl * kGroup + 4 * lane);
+    const int q0 = quant_code(v.x, s, rs), q1 = quant_code(v.y, s, rs);
+    const int q2 = quant_code(v.z, s, rs), q3 = quant_code(v.w, s, rs);
+    reinterpret_cast<uint32_t *>(xq + m * K + g * kGroup)[lane] =
+        (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
+        ((uint32_t)(q3 & 0xff) << 24);
+    int sum = q0 + q1 + q2 + q3;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (xsum && lane == 0) xsum[m * G + g] = sum;
+  }
+}
+
 // p with K = p or K = 28 p (p a power of two), or 0
 int block_length(int64_t K) {
   auto pow2 = [](int64_t v) { return v > 0 && (v & (v - 1)) == 0; };
@@ -221,6 +359,30 @@ cudaError_t launch_hadamard_quantize(const uint16_t *x, int64_t M, int64_t K, in
   int lp = 0;
   while ((1 << lp) < p) ++lp;
   const float norm = (float)(1.0 / sqrt((double)K));
+  if (K == 28 * 512 && M <= hd::kClusterMaxM) {
+    // decode sizes: a cluster of 7 CTAs per token
+    auto kern = hd::hadamard_quantize_cluster_kernel;
+    constexpr int smem = (int)sizeof(hd::ClusterSmem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(hd::kClusterCtas, (unsigned)M);
+    cfg.blockDim = dim3(hd::kCThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = hd::kClusterCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, kern, x, norm, xq, xs, xsum);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)K * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(hd::hadamard_quantize_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
