@@ -168,15 +168,31 @@ __host__ __device__ constexpr int smem_total(int mode, int bt, int stages) {
          16;
 }
 
-// d = a * b + c on float pairs (one packed f32x2 instruction).
-__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1,
-                                     float c0, float c1) {
-  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
-      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
-      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+// Float pairs in 64-bit registers and the packed f32x2 operations on them.
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
 }
+__device__ __forceinline__ uint64_t pack_i2(int lo, int hi) {  // the bit patterns
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack_f2(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add_f2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma_f2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 
 // XS: the kernel forms the tokens' group sums itself (no caller xsum).
 template <int MODE, int BT, bool ACTG, bool DEBUG, bool SPLIT, bool XS>
@@ -499,9 +515,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
       const TileCoord tc = tile_coord<BT, SPLIT>(p, tile);
       const int n = tc.n0 + row, m0 = tc.m0;
-      float acc[COLS];
+      // running sums of the tile row, as float pairs in 64-bit registers (the
+      // packed fma's operands, so no pair is assembled per instruction)
+      uint64_t acc2[COLS / 2];
 #pragma unroll
-      for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < COLS / 2; ++j) acc2[j] = 0ull;
       for (int g = tc.g0; g < tc.g1; ++g, ++it) {
         if (!ok) continue;  // after a give-up: no more waits, but every tile still arrives below
         const int cs = it % CS, b = it % NACC;
@@ -534,30 +552,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 p.S[((int64_t)m * p.N + n) * p.G + g] = (int)d[j] + cv[c + j] - (int)kMagicI;
             }
           } else {
+            const uint64_t nm = pack_f2(-kMagicF, -kMagicF);
+            const uint64_t sg2 = pack_f2(sg, sg);
 #pragma unroll
             for (int j = 0; j < CH; j += 4) {
               const int4 c4 = *reinterpret_cast<const int4 *>(cv + c + j);
               // 1.5 * 2^23 + exact group sum, as a float, minus the magic
-              float f0 = __int_as_float((int)d[j] + c4.x), f1 = __int_as_float((int)d[j + 1] + c4.y);
-              float f2 = __int_as_float((int)d[j + 2] + c4.z), f3 = __int_as_float((int)d[j + 3] + c4.w);
-              f32x2_add(f0, f1, f0, f1, -kMagicF, -kMagicF);
-              f32x2_add(f2, f3, f2, f3, -kMagicF, -kMagicF);
-              float s0 = sg, s1 = sg, s2 = sg, s3 = sg;
+              uint64_t f01 = pack_i2((int)d[j] + c4.x, (int)d[j + 1] + c4.y);
+              uint64_t f23 = pack_i2((int)d[j + 2] + c4.z, (int)d[j + 3] + c4.w);
+              f01 = add_f2(f01, nm);
+              f23 = add_f2(f23, nm);
+              uint64_t s01 = sg2, s23 = sg2;
               if (ACTG) {
                 const float4 x4 = *reinterpret_cast<const float4 *>(xv + c + j);
-                s0 *= x4.x;
-                s1 *= x4.y;
-                s2 *= x4.z;
-                s3 *= x4.w;
+                s01 = pack_f2(sg * x4.x, sg * x4.y);
+                s23 = pack_f2(sg * x4.z, sg * x4.w);
               }
-              fma2(acc[c + j], acc[c + j + 1], f0, f1, s0, s1, acc[c + j], acc[c + j + 1]);
-              fma2(acc[c + j + 2], acc[c + j + 3], f2, f3, s2, s3, acc[c + j + 2], acc[c + j + 3]);
+              acc2[(c + j) / 2] = fma_f2(f01, s01, acc2[(c + j) / 2]);
+              acc2[(c + j) / 2 + 1] = fma_f2(f23, s23, acc2[(c + j) / 2 + 1]);
             }
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&emptyC[cs]);
       }
+      float acc[COLS];
+#pragma unroll
+      for (int j = 0; j < COLS / 2; ++j) unpack_f2(acc2[j], acc[2 * j], acc[2 * j + 1]);
       if constexpr (SPLIT && !DEBUG) {
         // this range's partial sums of the warp's sub-block (rows of its lane
         // quarter, its columns), then one arrival per warp; the last of the
