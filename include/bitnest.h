@@ -48,10 +48,11 @@ extern "C" {
 /* Kernel family for bitnest_linear_path. */
 #define BITNEST_PATH_AUTO 0 /* the library picks (see bitnest_select_path)          */
 #define BITNEST_PATH_GEMV 1 /* decode GEMV (planes streamed by TMA, integer
-                               mma.sync group sums), M <= BITNEST_GEMV_MAX_M */
+                               mma.sync group sums), M <= BITNEST_GEMV_MAX_M
+                               (<= 8 where K is not a multiple of 1024) */
 #define BITNEST_PATH_TC 2   /* tcgen05 kind::i8 tensor-core GEMM, any M              */
 
-#define BITNEST_GEMV_MAX_M 8 /* largest M the GEMV kernels are built for */
+#define BITNEST_GEMV_MAX_M 16 /* largest M the GEMV kernels are built for */
 
 /* May be OR-ed into the `path` of bitnest_linear_path: the layer kernel is
  * launched with programmatic dependent launch and starts streaming hi, lo and
@@ -236,8 +237,9 @@ int bitnest_linear(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_
                    void *stream);
 
 /* bitnest_linear with an explicit kernel family (BITNEST_PATH_*, optionally
- * OR-ed with BITNEST_PATH_OVERLAP).  PATH_GEMV requires M <= BITNEST_GEMV_MAX_M
- * (else BITNEST_ERR_UNSUPPORTED_SHAPE). */
+ * OR-ed with BITNEST_PATH_OVERLAP).  PATH_GEMV requires M <= BITNEST_GEMV_MAX_M,
+ * and M <= 8 where K is not a multiple of 1024, and the tokens' codes must fit
+ * the kernel's shared memory (else BITNEST_ERR_UNSUPPORTED_SHAPE). */
 int bitnest_linear_path(int mode, const uint8_t *hi, const uint8_t *lo, const uint16_t *scale,
                         const int8_t *xq, const float *xscale, const int32_t *xsum, int64_t M,
                         int64_t N, int64_t K, float *y, int act_group, const uint16_t *bias,

@@ -50,7 +50,10 @@ def test_select_path():
     assert bn.select_path(bn.DRAFT, 1, 4096, 4096) == bn.PATH_GEMV
     assert bn.select_path(bn.TARGET, 4, 14336, 4096) == bn.PATH_GEMV
     assert bn.select_path(bn.TARGET, 8, 4096, 14336) == bn.PATH_GEMV
-    assert bn.select_path(bn.TARGET, 9, 4096, 4096) == bn.PATH_TC
+    assert bn.select_path(bn.TARGET, 9, 4096, 4096) == bn.PATH_GEMV  # two token blocks
+    assert bn.select_path(bn.TARGET, 16, 14336, 4096) == bn.PATH_GEMV
+    assert bn.select_path(bn.TARGET, 17, 4096, 4096) == bn.PATH_TC
+    assert bn.select_path(bn.TARGET, 9, 4096, 14336) == bn.PATH_TC  # codes too large to stage
     assert bn.select_path(bn.TARGET, 2048, 4096, 4096) == bn.PATH_TC
 
 

@@ -105,9 +105,11 @@ def test_quantize_bit_exact(M, K, act_group):
 # ------------------------------------------------------------ group sums
 SMALL = [(1, 1, 128), (1, 37, 1024), (2, 64, 1152), (3, 5, 256), (4, 512, 1024),
          (5, 33, 384), (6, 17, 2048), (7, 9, 4224), (8, 130, 1024)]
+# two 8-token column blocks of the TMA GEMV's MMA (K a multiple of 1024)
+WIDE = [(9, 70, 1024), (12, 33, 2048), (16, 130, 1024), (13, 2500, 4096), (16, 300, 4096)]
 
 
-@pytest.mark.parametrize("M,N,K", SMALL)
+@pytest.mark.parametrize("M,N,K", SMALL + WIDE)
 @pytest.mark.parametrize("mode", [0, 1])
 def test_gemv_group_sums_bit_exact(M, N, K, mode):
     p = Problem(M, N, K, seed=M * 7 + N)
@@ -118,7 +120,7 @@ def test_gemv_group_sums_bit_exact(M, N, K, mode):
 
 
 # ---------------------------------------------------------------- outputs
-@pytest.mark.parametrize("M,N,K", SMALL + [(4, 300, 14336), (1, 1024, 4096)])
+@pytest.mark.parametrize("M,N,K", SMALL + WIDE + [(4, 300, 14336), (1, 1024, 4096)])
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("act_group", [0, 128])
 def test_gemv_output(M, N, K, mode, act_group):
@@ -133,7 +135,7 @@ def test_gemv_bias():
         assert oracle.max_normalised_error(p.y_gpu(mode, bn.PATH_GEMV), p.y_ref(mode)) <= TOL
 
 
-@pytest.mark.parametrize("M", [1, 4, 8])
+@pytest.mark.parametrize("M", [1, 4, 8, 11, 16])
 def test_draft_equals_target_when_lo_is_eight(M):
     p = Problem(M, 257, 2048, seed=3, lo_eight=True)
     yd = p.y_gpu(0, bn.PATH_GEMV)
@@ -186,7 +188,8 @@ def test_llama3_projection_decode_sampled(name):
         assert np.array_equal(S[:, rows, :], oracle.group_sums(mode, hi_rows, lo_rows, q, K))
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (4, 1000, 2048), (3, 17, 14336), (8, 64, 1024)])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (4, 1000, 2048), (3, 17, 14336), (8, 64, 1024),
+                                   (16, 1000, 4096)])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_gemv_overlap_launch(M, N, K, mode):
     """Programmatic dependent launch after the quantiser gives the same result."""

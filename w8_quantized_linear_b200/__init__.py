@@ -22,7 +22,7 @@ PATH_AUTO = 0
 PATH_GEMV = 1
 PATH_TC = 2
 PATH_OVERLAP = 0x100  # OR into path: stream the weights before the previous kernel ends
-GEMV_MAX_M = 8
+GEMV_MAX_M = 16
 GROUP = 128
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

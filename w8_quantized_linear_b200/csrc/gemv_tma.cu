@@ -49,7 +49,7 @@ constexpr int kStepCols = 4096;                        // columns per stage = 32
 constexpr int kSegs = kStepCols / 256;                 // 128-byte plane segments per row
 constexpr int kPlaneBytes = kRows * kStepCols / 2;     // 32 KB: one TMA box per plane
 constexpr int kMaxStages = 8;
-constexpr int kRedSlots = 4;  // row blocks whose partial sums can be in flight
+constexpr int kRedSlots = 4;  // row blocks whose partial sums can be in flight (2 for 16 slots)
 // Weight bytes the producer issues (per CTA) before the activations are
 // loaded: the stream starts while the preceding kernel runs, yet the memory
 // queues are short again when the consumers' activation loads go out (two
@@ -79,12 +79,18 @@ __host__ __device__ inline int scale_pitch(int G) { return 8 * (((G + 7) / 8) | 
 // staged activations [M][2][Cp] x 16 B, group sums [Gp][8], group act. scales
 // [Gp][8], the CTA's group scales [nb * 16][pitch] fp16, partial-sum slots
 // [kRedSlots][warps][128] and their counters
+// token slots of the MMA's N side: one 8-column block up to 8 tokens, two
+// up to 16 (then two partial-sum slots instead of four: the staged codes
+// take the shared memory)
+__host__ __device__ constexpr int token_slots(int M) { return M > 8 ? 16 : 8; }
+__host__ __device__ constexpr int red_slots(int M) { return M > 8 ? 2 : kRedSlots; }
+
 __host__ __device__ inline int fixed_bytes(int M, int K, bool actg, int nb) {
   const int nks = (K + kStepCols - 1) / kStepCols;
   const int Cp = nks * (kStepCols / 32), Gp = nks * (kStepCols / kGroup);
-  const int G = K / kGroup;
-  int o = M * Cp * 32 + Gp * 32 + (actg ? Gp * 32 : 0) + (nb * kRows * scale_pitch(G) * 2 + 15) / 16 * 16 +
-          kRedSlots * kConsumerWarps * 128 * 4;
+  const int G = K / kGroup, TS = token_slots(M);
+  int o = M * Cp * 32 + Gp * TS * 4 + (actg ? Gp * TS * 4 : 0) +
+          (nb * kRows * scale_pitch(G) * 2 + 15) / 16 * 16 + red_slots(M) * kConsumerWarps * 16 * TS * 4;
   return (o + 1023) / 1024 * 1024;
 }
 
@@ -140,19 +146,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int OFF = CodeOffset<MODE>::value;
   constexpr int STAGE = stage_bytes(MODE);
   constexpr int GS = kStepCols / kGroup;  // groups per stage (32)
+  constexpr int TS = token_slots(M);      // token slots: 8 or 16
+  constexpr int NTB = TS / 8;             // 8-token column blocks of the MMA
+  constexpr int RED = 16 * TS;            // partial sums of a row block per warp
+  constexpr int RS = red_slots(M);        // partial-sum slots in flight
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   const int Cp = p.Cp, Gp = p.Gp, G = p.G, S = p.stages;
   uint4 *xs4 = reinterpret_cast<uint4 *>(smem);                    // [M][2][Cp]
-  int32_t *sr = reinterpret_cast<int32_t *>(smem + M * Cp * 32);   // [Gp][8] group sums
-  float *sxg = reinterpret_cast<float *>(sr + Gp * 8);             // [Gp][8] group act. scales
+  int32_t *sr = reinterpret_cast<int32_t *>(smem + M * Cp * 32);   // [Gp][TS] group sums
+  float *sxg = reinterpret_cast<float *>(sr + Gp * TS);            // [Gp][TS] group act. scales
   const int nb = (p.NB - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   const int sp = scale_pitch(G);
-  __half *ssc = reinterpret_cast<__half *>(sxg + (ACTG ? Gp * 8 : 0));  // [nb * 16][sp]
+  __half *ssc = reinterpret_cast<__half *>(sxg + (ACTG ? Gp * TS : 0));  // [nb * 16][sp]
   float *red = reinterpret_cast<float *>(
-      reinterpret_cast<uint8_t *>(ssc) + (nb * kRows * sp * 2 + 15) / 16 * 16);  // [slots][warps][128]
+      reinterpret_cast<uint8_t *>(ssc) + (nb * kRows * sp * 2 + 15) / 16 * 16);  // [slots][warps][RED]
   uint8_t *ring = smem + fixed_bytes(M, p.K, ACTG, nb);            // 1024-aligned stages
   uint64_t *full = reinterpret_cast<uint64_t *>(ring + S * STAGE);
   uint64_t *empty = full + kMaxStages;
@@ -186,35 +196,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gid = lane >> 2, tig = lane & 3;
     const int r0 = perm_row(gid), r1 = r0 + 8;
     const int t0 = 2 * tig;
-    float xt0 = 0.0f, xt1 = 0.0f;
-    if (!ACTG) {
-      xt0 = t0 < M ? __ldg(p.xscale + t0) : 0.0f;
-      xt1 = t0 + 1 < M ? __ldg(p.xscale + t0 + 1) : 0.0f;
-    }
-    for (int k = 0; k < nb; ++k) {
-      const int slot = k % kRedSlots;
-      if (!mbar_wait_warp(&part_full[slot], (k / kRedSlots) & 1)) return;
-      const float *rb = red + slot * (kConsumerWarps * 128);
-      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float xt[NTB][2];  // token scales of tokens t0, t0 + 1 of each column block
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float4 pv = *reinterpret_cast<const float4 *>(rb + w * 128 + lane * 4);
-        v[0] += pv.x;
-        v[1] += pv.y;
-        v[2] += pv.z;
-        v[3] += pv.w;
+    for (int b = 0; b < NTB; ++b)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int tk = 8 * b + t0 + e;
+        xt[b][e] = (!ACTG && tk < M) ? __ldg(p.xscale + tk) : 0.0f;
       }
+    for (int k = 0; k < nb; ++k) {
+      const int slot = k % RS;
+      if (!mbar_wait_warp(&part_full[slot], (k / RS) & 1)) return;
+      const float *rb = red + slot * (kConsumerWarps * RED);
       const int row0 = ((int)blockIdx.x + k * (int)gridDim.x) * kRows;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int tk = t0 + (i & 1);
-        const int n = row0 + ((i >> 1) ? r1 : r0);
-        if (tk < M && n < p.N) {
-          float out = v[i];
-          if (!ACTG) out *= (i & 1) ? xt1 : xt0;
-          if (MODE) out *= 0.0625f;
-          if (p.bias) out += __half2float(__ushort_as_half(__ldg(p.bias + n)));
-          p.y[(int64_t)tk * p.N + n] = out;
+      for (int b = 0; b < NTB; ++b) {
+        float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float4 pv = *reinterpret_cast<const float4 *>(rb + w * RED + b * 128 + lane * 4);
+          v[0] += pv.x;
+          v[1] += pv.y;
+          v[2] += pv.z;
+          v[3] += pv.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tk = 8 * b + t0 + (i & 1);
+          const int n = row0 + ((i >> 1) ? r1 : r0);
+          if (tk < M && n < p.N) {
+            float out = v[i];
+            if (!ACTG) out *= xt[b][i & 1];
+            if (MODE) out *= 0.0625f;
+            if (p.bias) out += __half2float(__ushort_as_half(__ldg(p.bias + n)));
+            p.y[(int64_t)tk * p.N + n] = out;
+          }
         }
       }
       __syncwarp();
@@ -276,14 +292,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_wait();  // the activations are written by the preceding kernel
   const int C = p.K / 32;
   // token slots M..7 of the group sums (the MMA's unused columns) are zero
-  if constexpr (M < 8)
-    for (int i = threadIdx.x; i < Gp * (8 - M); i += NT) sr[(i / (8 - M)) * 8 + M + i % (8 - M)] = 0;
+  if constexpr (M < TS)
+    for (int i = threadIdx.x; i < Gp * (TS - M); i += NT)
+      sr[(i / (TS - M)) * TS + M + i % (TS - M)] = 0;
   // activations (and per-group activation scales): every load of this
   // thread first (one round trip), then the permuted stores and the group
   // sums, formed here from the codes themselves
   constexpr int XB = 8;  // activation items per batch
   constexpr int RB = 4;  // activation-scale items per batch
-  for (int bx = 0, br = 0; bx < M * Cp || (ACTG && br < Gp * 8); bx += XB * NT, br += RB * NT) {
+  for (int bx = 0, br = 0; bx < M * Cp || (ACTG && br < Gp * TS); bx += XB * NT, br += RB * NT) {
     uint4 va[XB], vb[XB];
     float xv[RB];
 #pragma unroll
@@ -304,8 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int u = 0; u < RB; ++u) {
         const int i = br + threadIdx.x + u * NT;
-        const int g = i >> 3, m = i & 7;
-        const bool in = i < Gp * 8 && m < M && g < G;
+        const int g = i / TS, m = i % TS;
+        const bool in = i < Gp * TS && m < M && g < G;
         xv[u] = in ? __ldg(p.xscale + m * G + g) : 0.0f;
       }
     }
@@ -336,14 +353,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         xs4[(m * 2 + 0) * Cp + c] = make_uint4(e[0], o[0], e[1], o[1]);
         xs4[(m * 2 + 1) * Cp + c] = make_uint4(e[2], o[2], e[3], o[3]);
-        if ((c & 3) == 0) sr[(c >> 2) * 8 + m] = r;  // group c / 4 of token m (0 past K)
+        if ((c & 3) == 0) sr[(c >> 2) * TS + m] = r;  // group c / 4 of token m (0 past K)
       }
     }
     if (ACTG) {
 #pragma unroll
       for (int u = 0; u < RB; ++u) {
         const int i = br + threadIdx.x + u * NT;
-        if (i < Gp * 8) sxg[i] = xv[u];
+        if (i < Gp * TS) sxg[i] = xv[u];
       }
     }
   }
@@ -365,7 +382,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   int it = 0;
   for (int k = 0; k < nb; ++k) {
     const int row0 = ((int)blockIdx.x + k * (int)gridDim.x) * kRows;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float acc[NTB][4];
+#pragma unroll
+    for (int b = 0; b < NTB; ++b)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[b][i] = 0.0f;
     for (int ks = 0; ks < p.nks && ok; ++ks, ++it) {
       uint2 sc_cur0 = make_uint2(0, 0), sc_cur1 = make_uint2(0, 0);
       if (!DEBUG) {  // this warp's four group scales of rows r0, r1
@@ -391,20 +412,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           l0 = *reinterpret_cast<const uint4 *>(st + kPlaneBytes + off0);
           l1 = *reinterpret_cast<const uint4 *>(st + kPlaneBytes + off1);
         }
-        // activations of token gid, 32-column chunk 4g + tig, permuted even/odd
-        uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
-        if (gid < M) {
-          const int c = g * 4 + tig;
-          xa = xs4[(gid * 2 + 0) * Cp + c];
-          xb = xs4[(gid * 2 + 1) * Cp + c];
-        }
+        // activations of tokens gid (and gid + 8), 32-column chunk 4g + tig,
+        // permuted even/odd: the MMA's B operand of each 8-token column block
+        uint32_t xe[NTB][4], xo[NTB][4];
         // the accumulator starts at -offset * sum(q) of the group: the MMA
         // result is the exact group sum of q * weight code
-        const int2 rr = *reinterpret_cast<const int2 *>(sr + g * 8 + tok0);
-        int d[4] = {-OFF * rr.x, -OFF * rr.y, -OFF * rr.x, -OFF * rr.y};
+        int d[NTB][4];
+#pragma unroll
+        for (int b = 0; b < NTB; ++b) {
+          uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+          const int tk = 8 * b + gid;
+          if (tk < M) {
+            const int c = g * 4 + tig;
+            xa = xs4[(tk * 2 + 0) * Cp + c];
+            xb = xs4[(tk * 2 + 1) * Cp + c];
+          }
+          xe[b][0] = xa.x; xe[b][1] = xa.z; xe[b][2] = xb.x; xe[b][3] = xb.z;
+          xo[b][0] = xa.y; xo[b][1] = xa.w; xo[b][2] = xb.y; xo[b][3] = xb.w;
+          const int2 rr = *reinterpret_cast<const int2 *>(sr + g * TS + 8 * b + tok0);
+          d[b][0] = -OFF * rr.x;
+          d[b][1] = -OFF * rr.y;
+          d[b][2] = -OFF * rr.x;
+          d[b][3] = -OFF * rr.y;
+        }
         const uint32_t hw0[4] = {h0.x, h0.y, h0.z, h0.w}, hw1[4] = {h1.x, h1.y, h1.z, h1.w};
         const uint32_t lw0[4] = {l0.x, l0.y, l0.z, l0.w}, lw1[4] = {l1.x, l1.y, l1.z, l1.w};
-        const uint32_t xe[4] = {xa.x, xa.z, xb.x, xb.z}, xo[4] = {xa.y, xa.w, xb.y, xb.w};
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {  // 4 x K=32 columns of the group
           uint32_t a[4];
@@ -419,30 +451,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             a[2] = (hw0[jj] & 0xF0F0F0F0u) | ((lw0[jj] >> 4) & 0x0F0F0F0Fu);
             a[3] = (hw1[jj] & 0xF0F0F0F0u) | ((lw1[jj] >> 4) & 0x0F0F0F0Fu);
           }
-          mma_u8s8(d, a, xe[jj], xo[jj], d);
+#pragma unroll
+          for (int b = 0; b < NTB; ++b) mma_u8s8(d[b], a, xe[b][jj], xo[b][jj], d[b]);
         }
         if (DEBUG) {
           const int n0 = row0 + r0, n1 = row0 + r1;
           if (g < G) {
-            if (tok0 < M && n0 < p.N) p.S[((int64_t)tok0 * p.N + n0) * G + g] = d[0];
-            if (tok1 < M && n0 < p.N) p.S[((int64_t)tok1 * p.N + n0) * G + g] = d[1];
-            if (tok0 < M && n1 < p.N) p.S[((int64_t)tok0 * p.N + n1) * G + g] = d[2];
-            if (tok1 < M && n1 < p.N) p.S[((int64_t)tok1 * p.N + n1) * G + g] = d[3];
+#pragma unroll
+            for (int b = 0; b < NTB; ++b) {
+              const int t0 = 8 * b + tok0, t1 = 8 * b + tok1;
+              if (t0 < M && n0 < p.N) p.S[((int64_t)t0 * p.N + n0) * G + g] = d[b][0];
+              if (t1 < M && n0 < p.N) p.S[((int64_t)t1 * p.N + n0) * G + g] = d[b][1];
+              if (t0 < M && n1 < p.N) p.S[((int64_t)t0 * p.N + n1) * G + g] = d[b][2];
+              if (t1 < M && n1 < p.N) p.S[((int64_t)t1 * p.N + n1) * G + g] = d[b][3];
+            }
           }
         } else {
           const float s0 = half_bits_to_float(q < 2 ? sc_cur0.x : sc_cur0.y, q & 1);
           const float s1 = half_bits_to_float(q < 2 ? sc_cur1.x : sc_cur1.y, q & 1);
-          float x0 = 1.0f, x1 = 1.0f;
-          if (ACTG) {
-            const float2 xg = *reinterpret_cast<const float2 *>(sxg + g * 8 + tok0);
-            x0 = xg.x;
-            x1 = xg.y;
+#pragma unroll
+          for (int b = 0; b < NTB; ++b) {
+            float x0 = 1.0f, x1 = 1.0f;
+            if (ACTG) {
+              const float2 xg = *reinterpret_cast<const float2 *>(sxg + g * TS + 8 * b + tok0);
+              x0 = xg.x;
+              x1 = xg.y;
+            }
+            // |d| < 2^24: the conversions are exact
+            acc[b][0] = fmaf((float)d[b][0], ACTG ? s0 * x0 : s0, acc[b][0]);
+            acc[b][1] = fmaf((float)d[b][1], ACTG ? s0 * x1 : s0, acc[b][1]);
+            acc[b][2] = fmaf((float)d[b][2], ACTG ? s1 * x0 : s1, acc[b][2]);
+            acc[b][3] = fmaf((float)d[b][3], ACTG ? s1 * x1 : s1, acc[b][3]);
           }
-          // |d| < 2^24: the conversions are exact
-          acc[0] = fmaf((float)d[0], ACTG ? s0 * x0 : s0, acc[0]);
-          acc[1] = fmaf((float)d[1], ACTG ? s0 * x1 : s0, acc[1]);
-          acc[2] = fmaf((float)d[2], ACTG ? s1 * x0 : s1, acc[2]);
-          acc[3] = fmaf((float)d[3], ACTG ? s1 * x1 : s1, acc[3]);
         }
       }
       __syncwarp();
@@ -450,12 +490,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!DEBUG && ok) {
       // deposit this warp's partial sums of the row block for the reducer
-      const int slot = k % kRedSlots;
-      if (k >= kRedSlots) ok = mbar_wait_warp(&slot_free[slot], ((k / kRedSlots) - 1) & 1);
+      const int slot = k % RS;
+      if (k >= RS) ok = mbar_wait_warp(&slot_free[slot], ((k / RS) - 1) & 1);
       if (ok) {
-        float *rb = red + slot * (kConsumerWarps * 128);
-        *reinterpret_cast<float4 *>(rb + warp * 128 + lane * 4) =
-            make_float4(acc[0], acc[1], acc[2], acc[3]);
+        float *rb = red + slot * (kConsumerWarps * RED);
+#pragma unroll
+        for (int b = 0; b < NTB; ++b)
+          *reinterpret_cast<float4 *>(rb + warp * RED + b * 128 + lane * 4) =
+              make_float4(acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&part_full[slot]);
       }
@@ -570,6 +612,14 @@ cudaError_t dispatch_m(const LinearArgs &a, cudaStream_t st) {
     BITNEST_GV_CASE(6)
     BITNEST_GV_CASE(7)
     BITNEST_GV_CASE(8)
+    BITNEST_GV_CASE(9)
+    BITNEST_GV_CASE(10)
+    BITNEST_GV_CASE(11)
+    BITNEST_GV_CASE(12)
+    BITNEST_GV_CASE(13)
+    BITNEST_GV_CASE(14)
+    BITNEST_GV_CASE(15)
+    BITNEST_GV_CASE(16)
     default: return cudaErrorInvalidValue;
   }
 #undef BITNEST_GV_CASE
@@ -579,7 +629,7 @@ cudaError_t dispatch_m(const LinearArgs &a, cudaStream_t st) {
 
 bool gemv_tma_supported(int64_t M, int64_t N, int64_t K) {
   // the scale rows are read as 32-bit words and G is a multiple of 8
-  if (M < 1 || M > 8 || N < 1 || K % 1024 != 0 || K > (1 << 20)) return false;
+  if (M < 1 || M > 16 || N < 1 || K % 1024 != 0 || K > (1 << 20)) return false;
   const int64_t NB = (N + gv::kRows - 1) / gv::kRows;
   const int sms = gv::num_sms();
   const int64_t per = (NB + sms - 1) / sms;
