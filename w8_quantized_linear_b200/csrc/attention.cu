@@ -306,6 +306,9 @@ __global__ void __launch_bounds__(kThreads, 2) nested_attention_kernel(
     const float c0 = __shfl_sync(0xffffffffu, corr, 8 * tig) * unit;
     const float c1 = __shfl_sync(0xffffffffu, corr, 8 * tig + 4) * unit;
     e_run = e_tile;
+    // the running maxima and the unit settle after a few tiles: then the
+    // output needs no rescaling
+    const bool rescale = __any_sync(0xffffffffu, c0 != 1.0f || c1 != 1.0f);
     // ------------------------------------------------ O^T += V^T P'^T
     uint32_t ev[4][2], od[4][2];  // tokens 2 tig, 2 tig + 1, 8 + 2 tig, 9 + 2 tig; bytes 0..7
 #pragma unroll
@@ -320,10 +323,12 @@ __global__ void __launch_bounds__(kThreads, 2) nested_attention_kernel(
       const uint32_t a1 = pair<MODE>(od[0][w], od[1][w], b);  // odd column
       const uint32_t a2 = pair<MODE>(ev[2][w], ev[3][w], b);  // tokens 8 + 2 tig, 9 + 2 tig
       const uint32_t a3 = pair<MODE>(od[2][w], od[3][w], b);
-      o[mt][0] *= c0;
-      o[mt][1] *= c1;
-      o[mt][2] *= c0;
-      o[mt][3] *= c1;
+      if (rescale) {
+        o[mt][0] *= c0;
+        o[mt][1] *= c1;
+        o[mt][2] *= c0;
+        o[mt][3] *= c1;
+      }
       mma_f16(o[mt], a0, a1, a2, a3, bh0, bh1);
       mma_f16(o[mt], a0, a1, a2, a3, bl0, bl1);
     }
